@@ -1,0 +1,99 @@
+/*
+ * wan_attn.h - C ABI of the B200 (sm_100a) full self-attention library for
+ * Wan-style video diffusion transformers.
+ *
+ * The operation.  Inside every DiT block of Wan, all tokens of the patchified
+ * video latent attend to all other tokens, bidirectionally:
+ *     O = softmax(Q K^T / sqrt(D)) V,
+ * non-causal and neither windowed nor masked.  Sources: "Wan 2.1: VBench
+ * 86.22% ..." (paper-podcast summary of the Wan report), section
+ * "干预与形式化" (the DiT's full spatio-temporal self-attention) and section
+ * "先看现象" (cost model C = L(alpha*b*s*h^2 + beta*b*s^2*h), non-causal
+ * attention with beta = 4 forward and 8 backward; the token count
+ * (1+T/4)(H/16)(W/16) of the VAE latent after the (1,2,2) patchify);
+ * "Wan: Open and Advanced Large-Scale Video Generative Models", section 5
+ * (attention is what grows with sequence length in training).
+ *
+ * Conventions shared by every call:
+ *   - Q, K, V, O (and dO, dQ, dK, dV) are bf16 tensors laid out [B, S, H, D],
+ *     contiguous, D fastest.  D must be 128.
+ *   - lse is fp32 [B, H, S]: lse[b,h,i] = ln sum_j exp(q_i . k_j / sqrt(D)).
+ *   - The softmax scale is fixed at 1/sqrt(D).  No mask, no dropout, no bias.
+ *   - Every pointer is a device pointer owned by the caller, 16-byte aligned.
+ *     The library allocates no memory.  Outputs may not overlap inputs.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     validate their arguments on the host, enqueue their kernels and return;
+ *     they do not synchronise.  On a validation failure nothing is enqueued.
+ *   - Kernels never spin without bound: every wait inside a kernel has a time
+ *     budget; when one runs out the kernel records WAN_ATTN_ERR_TIMEOUT in a
+ *     device status word and exits.  wan_attn_sync_status() reports it.
+ */
+#ifndef WAN_ATTN_H
+#define WAN_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WAN_ATTN_API __attribute__((visibility("default")))
+#else
+#define WAN_ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WAN_ATTN_OK = 0,
+    WAN_ATTN_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, overlap */
+    WAN_ATTN_ERR_UNSUPPORTED = 2,   /* D != 128 */
+    WAN_ATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed (launch, tensor map) */
+    WAN_ATTN_ERR_TIMEOUT = 4,       /* a kernel's bounded wait ran out (reported by sync_status) */
+    WAN_ATTN_ERR_WORKSPACE = 5      /* workspace pointer null or smaller than required */
+} wan_attn_status;
+
+/*
+ * Forward, bf16.
+ *   q, k, v : in,  bf16 [B, S, H, D]
+ *   o       : out, bf16 [B, S, H, D], rounded to nearest even from fp32
+ *   lse     : out, fp32 [B, H, S], natural-log log-sum-exp of the scaled
+ *             scores of each query row (the backward's input); not NULL.
+ *   B, S, H : >= 1, with B*S*H*D < 2^40;  D : must be 128.
+ * Accumulation is fp32 (scores, running max and sum, and O).  Returns
+ * WAN_ATTN_OK once the kernel is enqueued.
+ */
+WAN_ATTN_API int wan_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int S, int H, int D, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word:
+ * WAN_ATTN_OK, WAN_ATTN_ERR_TIMEOUT (a kernel's bounded wait ran out), or
+ * WAN_ATTN_ERR_CUDA if the synchronisation itself failed.
+ */
+WAN_ATTN_API int wan_attn_sync_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+WAN_ATTN_API const char* wan_attn_status_string(int status);
+
+/*
+ * Time budget, in nanoseconds, of every bounded wait inside the kernels
+ * launched after this call on this process (default 2e9 = 2 s; values
+ * below 1000 are raised to 1000).  Returns the previous budget.
+ */
+WAN_ATTN_API uint64_t wan_attn_set_wait_budget_ns(uint64_t ns);
+
+/*
+ * Self-test of the bounded-wait path: launches one small CTA that waits on a
+ * barrier nobody arrives at, with the given budget, then exits through the
+ * same give-up path the attention kernels use.  A following
+ * wan_attn_sync_status() returns WAN_ATTN_ERR_TIMEOUT.  No counterpart in the
+ * pages: it exists so failure detection can be tested without faulting a GPU.
+ */
+WAN_ATTN_API int wan_attn_selftest_wait_timeout(uint64_t budget_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WAN_ATTN_H */

@@ -1,0 +1,35 @@
+"""Helpers for the GPU parity tests: move the seeded host inputs to the device
+and measure errors against the oracle."""
+import numpy as np
+
+import synth
+
+
+def to_device(bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def bf16_to_f64(t):
+    """bf16 CUDA tensor -> fp64 numpy (exact)."""
+    import torch
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def errors(got, want):
+    """(max-abs error, relative Frobenius error)."""
+    d = got - want
+    return float(np.abs(d).max()), float(np.linalg.norm(d) / np.linalg.norm(want))
+
+
+def inputs_for(B, S, H, D=128, seed=0, with_do=False, q_mul=1.0):
+    shape = (B, S, H, D)
+    x = {"q": synth.make_tensor(shape, seed, synth.STREAM_Q),
+         "k": synth.make_tensor(shape, seed, synth.STREAM_K),
+         "v": synth.make_tensor(shape, seed, synth.STREAM_V)}
+    if q_mul != 1.0:
+        f = synth.bf16_bits_to_f32(x["q"]) * np.float32(q_mul)
+        x["q"] = synth.f64_to_bf16_bits(f.astype(np.float64))
+    if with_do:
+        x["do"] = synth.make_tensor(shape, seed, synth.STREAM_DO)
+    return x

@@ -1,0 +1,71 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry point
+the header declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "wan_attn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wan_attn_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def built():
+    from video_dit_full_b200 import build
+    return build.build()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("wan_attn_fwd", "wan_attn_sync_status", "wan_attn_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(built):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", built], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    # nothing else of ours leaks out of the shared object
+    ours = sorted(n for n in exported if n.startswith("wan"))
+    assert ours == declared_functions()
+
+
+def test_binding_covers_every_symbol(built):
+    from video_dit_full_b200 import wan_attn
+    assert sorted(n for n, _, _ in wan_attn.SIGNATURES) == declared_functions()
+    lib = wan_attn.lib()
+    for name in declared_functions():
+        assert getattr(lib, name)
+
+
+def test_host_side_validation_without_gpu(built):
+    from video_dit_full_b200 import wan_attn
+    lib = wan_attn.lib()
+    p = ctypes.c_void_p(0x10000)      # aligned fake addresses: never dereferenced on these paths
+    p2, p3, p4, p5 = (ctypes.c_void_p(0x10000 + i * 0x1000000) for i in range(1, 5))
+    INVALID, UNSUPPORTED = 1, 2
+    assert lib.wan_attn_fwd(None, p2, p3, p4, p5, 1, 128, 1, 128, None) == INVALID
+    assert lib.wan_attn_fwd(p, p2, p3, p4, None, 1, 128, 1, 128, None) == INVALID
+    assert lib.wan_attn_fwd(p, p2, p3, p4, p5, 0, 128, 1, 128, None) == INVALID
+    assert lib.wan_attn_fwd(p, p2, p3, p4, p5, 1, -5, 1, 128, None) == INVALID
+    assert lib.wan_attn_fwd(p, p2, p3, p4, p5, 1, 128, 1, 64, None) == UNSUPPORTED
+    odd = ctypes.c_void_p(0x10008)
+    assert lib.wan_attn_fwd(odd, p2, p3, p4, p5, 1, 128, 1, 128, None) == INVALID
+    # output overlapping an input
+    assert lib.wan_attn_fwd(p, p2, p3, p, p5, 1, 128, 1, 128, None) == INVALID
+    # lse overlapping o
+    assert lib.wan_attn_fwd(p, p2, p3, p4, ctypes.c_void_p(0x10000 + 3 * 0x1000000 + 64), 1, 128, 1, 128,
+                            None) == INVALID
+    assert lib.wan_attn_status_string(4) == b"a kernel wait ran out of time"
+    old = lib.wan_attn_set_wait_budget_ns(5)
+    assert lib.wan_attn_set_wait_budget_ns(old) == 1000

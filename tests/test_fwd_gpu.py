@@ -1,0 +1,108 @@
+"""Parity of the bf16 forward (wan_attn_fwd, through the C ABI) with the fp64 oracle.
+
+Bar (the workload's stated tolerance): on O, max-abs error <= 1e-2 and
+relative Frobenius error <= 5e-3.  The LSE is checked to 1e-3 absolute (fp32
+sums of exact bf16 products; the observed error is ~1e-6).
+
+Stress inputs outside the workloads (scores with std 8, where softmax is
+nearly one-hot and |O| reaches ~4) use a max-abs bound scaled by the output's
+magnitude: bf16 rounding of O and of P each contribute up to 2^-9 relative,
+so max-abs <= max(1e-2, 6e-3 * max|O|).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import bf16_to_f64, errors, inputs_for, to_device
+
+pytestmark = pytest.mark.gpu
+
+O_MAX_ABS, O_REL_FROB, LSE_MAX_ABS = 1e-2, 5e-3, 1e-3
+
+
+def run_fwd(x):
+    import torch
+    import video_dit_full_b200 as wa
+    q, k, v = (to_device(x[n]) for n in "qkv")
+    o, lse = wa.fwd(q, k, v)
+    wa.check_status()
+    return o, lse
+
+
+def check(x, rows=None, heads=None, scale_abs=False):
+    o, lse = run_fwd(x)
+    want_o, want_lse = oracle.attn_fwd(x["q"], x["k"], x["v"], rows=rows, heads=heads)
+    got_o = bf16_to_f64(o)
+    got_lse = lse.cpu().numpy().astype(np.float64)
+    if rows is not None:
+        got_o = got_o[:, rows]
+        got_lse = got_lse[:, :, rows]
+    if heads is not None:
+        got_o = got_o[:, :, heads]
+        got_lse = got_lse[:, heads]
+    assert np.all(np.isfinite(got_o)) and np.all(np.isfinite(got_lse))
+    max_abs, rel = errors(got_o, want_o)
+    lse_err = float(np.abs(got_lse - want_lse).max())
+    print(f"O max-abs {max_abs:.3e} rel-frob {rel:.3e}  LSE max-abs {lse_err:.3e}")
+    bound = max(O_MAX_ABS, 6e-3 * float(np.abs(want_o).max())) if scale_abs else O_MAX_ABS
+    assert max_abs <= bound and rel <= O_REL_FROB, (max_abs, rel, bound)
+    assert lse_err <= LSE_MAX_ABS, lse_err
+    return o, lse
+
+
+@pytest.mark.parametrize("B,S,H", [(1, 1, 1), (1, 2, 1), (2, 63, 2), (1, 64, 1), (1, 65, 3), (1, 127, 1),
+                                   (2, 128, 2), (1, 129, 1), (1, 255, 2), (1, 256, 1), (1, 257, 2),
+                                   (2, 300, 3), (1, 1000, 2), (3, 520, 1)])
+def test_fwd_ragged_shapes_full(B, S, H):
+    check(inputs_for(B, S, H, seed=S))
+
+
+def test_fwd_oracle_sized_workload_full():
+    w = synth.WORKLOADS["oracle_1280"]
+    check(synth.make_inputs(w))
+
+
+def test_fwd_large_scores_exercise_rescaling():
+    # scores with std 8: the running max moves many times and P is peaky
+    check(inputs_for(2, 700, 2, seed=11, q_mul=8.0), scale_abs=True)
+
+
+def test_fwd_increasing_scores_rescale_every_tile():
+    B, S, H, D = 1, 1500, 1, 128
+    u = np.ones(D) / np.sqrt(D) * 4.0
+    q = np.broadcast_to(u, (B, S, H, D))
+    ramp = (np.arange(S) / 40.0)[None, :, None, None]
+    k = ramp * np.broadcast_to(u, (B, S, H, D)) * np.sqrt(D) / 16.0   # s_ij = j / 40: the max rises along keys
+    v = np.random.default_rng(5).standard_normal((B, S, H, D))
+    x = {n: synth.f64_to_bf16_bits(a) for n, a in (("q", q), ("k", k), ("v", v))}
+    check(x, scale_abs=True)
+
+
+def test_fwd_is_deterministic():
+    x = inputs_for(1, 777, 3, seed=3)
+    o1, l1 = run_fwd(x)
+    o2, l2 = run_fwd(x)
+    assert bool((o1 == o2).all()) and bool((l1 == l2).all())
+
+
+def test_fwd_cfg_480p_sampled_rows():
+    w = synth.WORKLOADS["wan1.3b_480p_cfg"]
+    x = synth.make_inputs(w)
+    rows = synth.sample_rows(w.S, 256)
+    check(x, rows=rows)
+
+
+def test_fwd_14b_720p_sampled_rows():
+    w = synth.WORKLOADS["wan14b_720p"]
+    x = synth.make_inputs(w)
+    rows = synth.sample_rows(w.S, 256)
+    check(x, rows=rows)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    import video_dit_full_b200 as wa
+    wa.selftest_wait_timeout(2_000_000)          # 2 ms budget on a barrier nobody arrives at
+    assert wa.sync_status() == 4                  # WAN_ATTN_ERR_TIMEOUT
+    assert wa.sync_status() == 0                  # cleared
+    check(inputs_for(1, 200, 1, seed=1))          # the context is still usable

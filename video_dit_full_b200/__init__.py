@@ -1,0 +1,7 @@
+"""B200 (sm_100a) full spatio-temporal self-attention for Wan-style video DiTs.
+
+The computation lives in ``libwan_attn.so`` (hand-written CUDA for sm_100a,
+C ABI in ``include/wan_attn.h``); ``wan_attn`` is its ctypes binding.
+"""
+from .wan_attn import (WanAttnError, check_status, fwd, lib, selftest_wait_timeout,  # noqa: F401
+                       set_wait_budget_ns, sync_status)

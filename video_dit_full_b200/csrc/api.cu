@@ -1,0 +1,192 @@
+// C-ABI layer: argument validation, TMA tensor maps, launches, status word.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "../../include/wan_attn.h"
+#include "sm100_ptx.cuh"
+#include "wan_attn_internal.h"
+
+namespace wan {
+
+__device__ int g_device_status = 0;
+
+int* device_status_word() {
+    static std::mutex mu;
+    static int* addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_device_status) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int*>(a);
+    }
+    return addr[dev];
+}
+
+namespace {
+
+std::atomic<unsigned long long> g_wait_budget_ns{2000000000ull};
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map over a bf16 [B, S, H, D] tensor viewed as 4-D (D, H, S, B), box
+// (64 of D, 1 head, `box_tokens` tokens, 1 batch) with the 128-byte swizzle.
+// Coordinates past S read as zero.
+bool make_bshd_map(CUtensorMap* m, const void* base, int B, int S, int H, int D, int box_tokens) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_tokens, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Range {
+    uintptr_t lo, hi;
+};
+Range range_of(const void* p, size_t bytes) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return {a, a + bytes};
+}
+bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks common to every call.  Returns a wan_attn_status.
+int check_shape(int B, int S, int H, int D) {
+    if (B < 1 || S < 1 || H < 1 || D < 1) return WAN_ATTN_ERR_INVALID_ARG;
+    if (D != 128) return WAN_ATTN_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535) return WAN_ATTN_ERR_INVALID_ARG;       // grid y/z limits
+    const double n = double(B) * S * H * D;
+    if (n >= double(1ull << 40)) return WAN_ATTN_ERR_INVALID_ARG;
+    return WAN_ATTN_OK;
+}
+
+}  // namespace
+
+int configure_smem(const void* kernel, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void*>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({dev, kernel})) return 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return -1;
+    done.insert({dev, kernel});
+    return 0;
+}
+
+unsigned long long wait_budget_ns() { return g_wait_budget_ns.load(); }
+
+// ---------------------------------------------------------------------------
+// bounded-wait self test: one warp waits on a barrier that nobody arrives at
+// ---------------------------------------------------------------------------
+__global__ void selftest_wait_kernel(unsigned long long budget_ns, int* status) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const WaitCtl wc{&abort_flag, budget_ns, status};
+    (void)wait_warp(b, 0, wc);     // gives up after budget_ns and records the timeout
+    __syncthreads();
+}
+
+}  // namespace wan
+
+using namespace wan;
+
+extern "C" {
+
+int wan_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S, int H, int D,
+                 void* stream) {
+    if (!q || !k || !v || !o || !lse) return WAN_ATTN_ERR_INVALID_ARG;
+    const int st = check_shape(B, S, H, D);
+    if (st != WAN_ATTN_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return WAN_ATTN_ERR_INVALID_ARG;
+    const size_t n = size_t(B) * S * H * D;
+    const Range rq = range_of(q, n * 2), rk = range_of(k, n * 2), rv = range_of(v, n * 2);
+    const Range ro = range_of(o, n * 2), rl = range_of(lse, size_t(B) * H * S * 4);
+    for (const Range& in : {rq, rk, rv})
+        if (overlaps(ro, in) || overlaps(rl, in)) return WAN_ATTN_ERR_INVALID_ARG;
+    if (overlaps(ro, rl)) return WAN_ATTN_ERR_INVALID_ARG;
+
+    CUtensorMap tq, tk, tv;
+    if (!make_bshd_map(&tq, q, B, S, H, D, 128) || !make_bshd_map(&tk, k, B, S, H, D, 128) ||
+        !make_bshd_map(&tv, v, B, S, H, D, 128))
+        return WAN_ATTN_ERR_CUDA;
+    FwdParams p;
+    p.o = o;
+    p.lse = lse;
+    p.B = B;
+    p.S = S;
+    p.H = H;
+    p.scale_log2 = static_cast<float>((1.0 / std::sqrt(double(D))) * 1.4426950408889634);
+    p.wait_budget_ns = wait_budget_ns();
+    p.status = device_status_word();
+    if (!p.status) return WAN_ATTN_ERR_CUDA;
+    return launch_fwd(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
+}
+
+int wan_attn_sync_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WAN_ATTN_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpyFromSymbol(&h, g_device_status, sizeof(int)) != cudaSuccess) return WAN_ATTN_ERR_CUDA;
+    if (h != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return WAN_ATTN_ERR_CUDA;
+    }
+    return h;
+}
+
+const char* wan_attn_status_string(int status) {
+    switch (status) {
+        case WAN_ATTN_OK: return "ok";
+        case WAN_ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case WAN_ATTN_ERR_UNSUPPORTED: return "unsupported (head dim must be 128)";
+        case WAN_ATTN_ERR_CUDA: return "CUDA error";
+        case WAN_ATTN_ERR_TIMEOUT: return "a kernel wait ran out of time";
+        case WAN_ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+uint64_t wan_attn_set_wait_budget_ns(uint64_t ns) {
+    if (ns < 1000) ns = 1000;
+    return g_wait_budget_ns.exchange(ns);
+}
+
+int wan_attn_selftest_wait_timeout(uint64_t budget_ns, void* stream) {
+    if (budget_ns < 1000) budget_ns = 1000;
+    int* status = device_status_word();
+    if (!status) return WAN_ATTN_ERR_CUDA;
+    selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_ns, status);
+    return cudaGetLastError() == cudaSuccess ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,31 @@
+// Internal declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace wan {
+
+struct FwdParams {
+    void* o;                    // bf16 [B, S, H, 128]
+    float* lse;                 // fp32 [B, H, S], natural log
+    int B, S, H;
+    float scale_log2;           // (1 / sqrt(D)) * log2(e)
+    unsigned long long wait_budget_ns;
+    int* status;                // device status word (see wan_attn_sync_status)
+};
+
+// Device address of the status word on the current device (nullptr on failure).
+int* device_status_word();
+unsigned long long wait_budget_ns();
+
+// Sets the dynamic shared-memory limit of a kernel once per device.  0 on success.
+int configure_smem(const void* kernel, int bytes);
+
+int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+               cudaStream_t stream);
+
+}  // namespace wan

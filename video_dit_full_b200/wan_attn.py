@@ -1,0 +1,113 @@
+"""Thin ctypes binding of ``libwan_attn.so`` (the C ABI in ``include/wan_attn.h``).
+
+Argument marshalling only: torch tensors are checked for dtype, device, shape
+and contiguity, and their device pointers and the current CUDA stream are
+passed to the library, which runs every step of the computation in its own
+kernels.  There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libwan_attn.so")
+
+STATUS = {0: "WAN_ATTN_OK", 1: "WAN_ATTN_ERR_INVALID_ARG", 2: "WAN_ATTN_ERR_UNSUPPORTED",
+          3: "WAN_ATTN_ERR_CUDA", 4: "WAN_ATTN_ERR_TIMEOUT", 5: "WAN_ATTN_ERR_WORKSPACE"}
+
+# (name, restype, argtypes) of every entry point the header declares
+_P, _I, _Z, _U64, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_void_p
+SIGNATURES = [
+    ("wan_attn_fwd", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P]),
+    ("wan_attn_sync_status", _I, [_P]),
+    ("wan_attn_status_string", ctypes.c_char_p, [_I]),
+    ("wan_attn_set_wait_budget_ns", _U64, [_U64]),
+    ("wan_attn_selftest_wait_timeout", _I, [_U64, _P]),
+]
+
+
+class WanAttnError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        self.status = status
+        super().__init__(f"{call} failed: {STATUS.get(status, status)}")
+
+
+_lib = None
+
+
+def lib():
+    """Load the library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m video_dit_full_b200.build` "
+                               "(there is no fallback implementation)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(call: str, status: int):
+    if status != 0:
+        raise WanAttnError(call, status)
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_bshd(name, t, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B, S, H, D] tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def fwd(q, k, v, o=None, lse=None, stream=None):
+    """O, LSE = attention(q, k, v) through ``wan_attn_fwd``; outputs allocated if not given."""
+    import torch
+    _check_bshd("q", q)
+    B, S, H, D = q.shape
+    _check_bshd("k", k, q.shape)
+    _check_bshd("v", v, q.shape)
+    if o is None:
+        o = torch.empty_like(q)
+    _check_bshd("o", o, q.shape)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, S) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, S] tensor")
+    _check("wan_attn_fwd", lib().wan_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                              lse.data_ptr(), B, S, H, D, _stream_ptr(stream)))
+    return o, lse
+
+
+def sync_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return lib().wan_attn_sync_status(_stream_ptr(stream))
+
+
+def check_status(stream=None):
+    _check("wan_attn_sync_status", sync_status(stream))
+
+
+def set_wait_budget_ns(ns: int) -> int:
+    return lib().wan_attn_set_wait_budget_ns(ns)
+
+
+def selftest_wait_timeout(budget_ns: int, stream=None):
+    _check("wan_attn_selftest_wait_timeout", lib().wan_attn_selftest_wait_timeout(budget_ns, _stream_ptr(stream)))
