@@ -288,7 +288,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wan14b_720p", choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--cpu-rows", type=int, default=64, help="query rows per head timed for cpu_baseline")
+    ap.add_argument("--cpu-rows", type=int, default=128, help="query rows per head timed for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="query rows per head per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -67,6 +67,34 @@ WAN_ATTN_API int wan_attn_fwd(const void* q, const void* k, const void* v, void*
                  int B, int S, int H, int D, void* stream);
 
 /*
+ * Bytes of device workspace wan_attn_bwd needs for these sizes: an fp32 dQ
+ * accumulator [B, S, H, D] followed by fp32 D_i = rowsum(dO * O) [B, H, S],
+ * each starting on a 256-byte boundary.  Returns 0 if the sizes are invalid.
+ */
+WAN_ATTN_API size_t wan_attn_bwd_workspace_size(int B, int S, int H, int D);
+
+/*
+ * Backward, bf16: gradients of sum(O * dO) for O = attention(Q, K, V).
+ *   q, k, v : in,  bf16 [B, S, H, D] (the forward's inputs)
+ *   o       : in,  bf16 [B, S, H, D] (the forward's output)
+ *   dO      : in,  bf16 [B, S, H, D]
+ *   lse     : in,  fp32 [B, H, S] written by wan_attn_fwd for the same inputs
+ *   dq, dk, dv : out, bf16 [B, S, H, D], rounded to nearest even
+ *   workspace, workspace_bytes : caller-owned device memory, 256-byte aligned,
+ *             at least wan_attn_bwd_workspace_size(B, S, H, D) bytes
+ *             (else WAN_ATTN_ERR_WORKSPACE).  Its contents on entry are
+ *             ignored; it must not overlap any other argument.
+ * The softmax matrix is recomputed from lse, never stored: P = exp(S/sqrt(D)
+ * - lse), dS = P * (dP - D), dV = P^T dO, dK = dS^T Q / sqrt(D), dQ = dS K /
+ * sqrt(D) (the non-causal backward of the cost model's beta = 8 term).
+ * dQ is accumulated in fp32 in the workspace across key tiles (atomic adds),
+ * so its low bits may differ between runs; dK and dV are deterministic.
+ */
+WAN_ATTN_API int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                              const float* lse, void* dq, void* dk, void* dv, int B, int S, int H, int D,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word:
  * WAN_ATTN_OK, WAN_ATTN_ERR_TIMEOUT (a kernel's bounded wait ran out), or
  * WAN_ATTN_ERR_CUDA if the synchronisation itself failed.

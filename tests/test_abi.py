@@ -69,3 +69,24 @@ def test_host_side_validation_without_gpu(built):
     assert lib.wan_attn_status_string(4) == b"a kernel wait ran out of time"
     old = lib.wan_attn_set_wait_budget_ns(5)
     assert lib.wan_attn_set_wait_budget_ns(old) == 1000
+
+
+def test_bwd_host_side_validation_without_gpu(built):
+    from video_dit_full_b200 import wan_attn
+    lib = wan_attn.lib()
+    ptr = [ctypes.c_void_p(0x100000 + i * 0x1000000) for i in range(11)]
+    q, k, v, o, do, lse, dq, dk, dv, ws = ptr[:10]
+    need = lib.wan_attn_bwd_workspace_size(1, 128, 2, 128)
+    assert need == 128 * 2 * 128 * 4 + 256 * 4
+    assert lib.wan_attn_bwd_workspace_size(1, 128, 2, 64) == 0
+    args = lambda **kw: [kw.get(n, d) for n, d in zip(
+        ["q", "k", "v", "o", "do", "lse", "dq", "dk", "dv", "B", "S", "H", "D", "ws", "wsb", "st"],
+        [q, k, v, o, do, lse, dq, dk, dv, 1, 128, 2, 128, ws, need, None])]
+    INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 5
+    assert lib.wan_attn_bwd(*args(do=None)) == INVALID
+    assert lib.wan_attn_bwd(*args(D=96)) == UNSUPPORTED
+    assert lib.wan_attn_bwd(*args(ws=None)) == WORKSPACE
+    assert lib.wan_attn_bwd(*args(wsb=need - 1)) == WORKSPACE
+    assert lib.wan_attn_bwd(*args(ws=ctypes.c_void_p(0x100000 + 9 * 0x1000000 + 16))) == WORKSPACE
+    assert lib.wan_attn_bwd(*args(dq=q)) == INVALID                 # output aliases an input
+    assert lib.wan_attn_bwd(*args(dk=dv)) == INVALID                # two outputs alias

@@ -70,6 +70,7 @@ Range range_of(const void* p, size_t bytes) {
 }
 bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Shape checks common to every call.  Returns a wan_attn_status.
 int check_shape(int B, int S, int H, int D) {
@@ -151,6 +152,58 @@ int wan_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
     return launch_fwd(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
+}
+
+size_t wan_attn_bwd_workspace_size(int B, int S, int H, int D) {
+    if (check_shape(B, S, H, D) != WAN_ATTN_OK) return 0;
+    const size_t n = size_t(B) * S * H * D;
+    return align256(n * 4) + align256(size_t(B) * H * S * 4);
+}
+
+int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int S, int H, int D, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return WAN_ATTN_ERR_INVALID_ARG;
+    const int st = check_shape(B, S, H, D);
+    if (st != WAN_ATTN_OK) return st;
+    for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(lse), static_cast<const void*>(dq),
+                            static_cast<const void*>(dk), static_cast<const void*>(dv)})
+        if (!aligned16(ptr)) return WAN_ATTN_ERR_INVALID_ARG;
+    const size_t need = wan_attn_bwd_workspace_size(B, S, H, D);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return WAN_ATTN_ERR_WORKSPACE;
+    const size_t n = size_t(B) * S * H * D;
+    const Range ins[] = {range_of(q, n * 2), range_of(k, n * 2), range_of(v, n * 2), range_of(o, n * 2),
+                         range_of(dO, n * 2), range_of(lse, size_t(B) * H * S * 4)};
+    const Range outs[] = {range_of(dq, n * 2), range_of(dk, n * 2), range_of(dv, n * 2),
+                          range_of(workspace, need)};
+    for (size_t a = 0; a < 4; ++a) {
+        for (const Range& in : ins)
+            if (overlaps(outs[a], in)) return WAN_ATTN_ERR_INVALID_ARG;
+        for (size_t c = a + 1; c < 4; ++c)
+            if (overlaps(outs[a], outs[c])) return WAN_ATTN_ERR_INVALID_ARG;
+    }
+
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_bshd_map(&tq, q, B, S, H, D, 128) || !make_bshd_map(&tk, k, B, S, H, D, 128) ||
+        !make_bshd_map(&tv, v, B, S, H, D, 128) || !make_bshd_map(&tdo, dO, B, S, H, D, 128))
+        return WAN_ATTN_ERR_CUDA;
+    BwdParams p;
+    p.lse = lse;
+    p.dq_acc = static_cast<float*>(workspace);
+    p.delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(n * 4));
+    p.dk = dk;
+    p.dv = dv;
+    p.B = B;
+    p.S = S;
+    p.H = H;
+    p.scale = static_cast<float>(1.0 / std::sqrt(double(D)));
+    p.scale_log2 = static_cast<float>((1.0 / std::sqrt(double(D))) * 1.4426950408889634);
+    p.wait_budget_ns = wait_budget_ns();
+    p.status = device_status_word();
+    if (!p.status) return WAN_ATTN_ERR_CUDA;
+    return launch_bwd(tq, tk, tv, tdo, p, o, dO, dq, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                          : WAN_ATTN_ERR_CUDA;
 }
 
 int wan_attn_sync_status(void* stream) {

@@ -1,0 +1,429 @@
+// bf16 backward of the Wan DiT full (non-causal) self-attention on sm_100a.
+//
+// The training step differentiates the same full spatio-temporal attention
+// ("Wan 2.1 ... paper-podcast summary", section "先看现象": beta = 8 for the
+// non-causal backward in the cost model).  With P = exp(S/sqrt(D) - lse),
+// D_i = rowsum(dO_i * O_i) and dS = P * (dP - D):
+//     dV = P^T dO,  dK = dS^T Q / sqrt(D),  dQ = dS K / sqrt(D),  dP = dO V^T.
+//
+// Three kernels:
+//   bwd_prep    D_i = sum_d dO_id O_id (fp32) and zeroing of the fp32 dQ accumulator.
+//   bwd_main    one CTA per 128-key tile of one (batch, head); K_j, V_j stay in
+//               shared memory while the CTA walks every 128-row Q tile i:
+//                 S^T = K Q_i^T, dP^T = V dO_i^T            (tcgen05, TMEM)
+//                 P^T = exp2(S^T c - lse_i log2 e)          (softmax warpgroup)
+//                 dV += P^T dO_i                            (A = P^T in TMEM)
+//                 dS^T = P^T (dP^T - D_i)  -> TMEM and smem (into dO_i's buffer)
+//                 dK += dS^T Q_i                            (A = dS^T in TMEM)
+//                 dQ_i^T = K^T dS^T  -> TMEM -> fp32 red.add into the accumulator
+//               P is recomputed from the forward's LSE; nothing of size S x S is stored.
+//   bwd_dq      dQ = bf16(accumulator / sqrt(D)).
+#include <cuda.h>
+
+#include "sm100_ptx.cuh"
+#include "wan_attn_internal.h"
+
+namespace wan {
+namespace bwd {
+
+constexpr int BM = 128;                  // keys per CTA (and queries per Q tile)
+constexpr int HD = 128;
+constexpr int TILE_BYTES = BM * HD * 2;  // 32 KB bf16 tile
+constexpr int HALF_BYTES = TILE_BYTES / 2;
+
+constexpr int OFF_K = 0;
+constexpr int OFF_V = OFF_K + TILE_BYTES;
+constexpr int OFF_Q = OFF_V + TILE_BYTES;          // 2 stages
+constexpr int OFF_DO = OFF_Q + 2 * TILE_BYTES;     // 2 stages (dS^T reuses the stage after dV)
+constexpr int OFF_VEC = OFF_DO + 2 * TILE_BYTES;   // per warp: 128 fp32 lse*log2(e), 128 fp32 D_i
+constexpr int VEC_BYTES = 2 * BM * 4;
+constexpr int OFF_BAR = OFF_VEC + 4 * VEC_BYTES;
+enum Bar { KV_FULL = 0, QDO_FULL = 1, QDO_EMPTY = 3, S_FULL = 5, DP_FULL = 6, P_READY = 7, DV_DONE = 8,
+           DS_READY = 9, DQ_FULL = 10, DQ_DRAINED = 11, FINAL = 12, DRAIN = 13, NBARS = 14 };
+constexpr int OFF_TMEM_SLOT = OFF_BAR + NBARS * 8;
+constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
+constexpr int SMEM_USED = OFF_ABORT + 8;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;
+constexpr int NTHREADS = 192;            // warps 0-3 softmax/gradients, 4 TMA, 5 MMA
+constexpr uint32_t TMEM_COLS = 512;      // S^T | dP^T | dV | dK
+constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
+constexpr float LOG2E = 1.4426950408889634f;
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 8 MMAs of K = 16 over a [128 rows][128 cols] bf16 tile pair, both K-major (K = the 128 columns).
+__device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, uint32_t idesc,
+                                           bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+        mma_f16_ss(d_tmem, sdesc_sw128(a_smem + off, 16, 1024), sdesc_sw128(b_smem + off, 16, 1024), idesc,
+                   (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+// A in TMEM (bf16, 128 x 128), B MN-major in shared memory: K = the 128 rows of the B tile.
+__device__ __forceinline__ void mma_ts_bmn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, uint32_t idesc,
+                                           bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_f16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc,
+                   (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// A and B both MN-major in shared memory, K = the 128 rows of both tiles.
+__device__ __forceinline__ void mma_ss_mn(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_f16_ss(d_tmem, sdesc_sw128(a_smem + kk * 2048, HALF_BYTES, 1024),
+                   sdesc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc, kk > 0 ? 1u : 0u);
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > budget_ns) break;
+    }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
+                const BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_addr);
+
+    const int warp = warp_id();
+    const int lane = lane_id();
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int kv0 = blockIdx.x * BM;
+    const int S = p.S;
+    const int nq = (S + BM - 1) / BM;
+
+    const uint32_t sK = base + OFF_K, sV = base + OFF_V, sQ = base + OFF_Q, sDO = base + OFF_DO;
+    const uint32_t bar0 = base + OFF_BAR;
+    auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
+    const WaitCtl wc{abort_flag, p.wait_budget_ns, p.status};
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(KV_FULL), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(QDO_FULL + s), 1);
+            mbar_init(bar(QDO_EMPTY + s), 1);
+        }
+        mbar_init(bar(S_FULL), 1);
+        mbar_init(bar(DP_FULL), 1);
+        mbar_init(bar(P_READY), BM);
+        mbar_init(bar(DV_DONE), 1);
+        mbar_init(bar(DS_READY), BM);
+        mbar_init(bar(DQ_FULL), 1);
+        mbar_init(bar(DQ_DRAINED), BM);
+        mbar_init(bar(FINAL), 1);
+        mbar_init(bar(DRAIN), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(base + OFF_TMEM_SLOT, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
+
+    if (warp == 4) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            tma_prefetch_desc(&tmq);
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+            tma_prefetch_desc(&tmdo);
+            mbar_arrive_expect_tx(bar(KV_FULL), 2 * TILE_BYTES);
+            tma_load_4d(sK, &tmk, bar(KV_FULL), 0, h, kv0, b);
+            tma_load_4d(sK + HALF_BYTES, &tmk, bar(KV_FULL), 64, h, kv0, b);
+            tma_load_4d(sV, &tmv, bar(KV_FULL), 0, h, kv0, b);
+            tma_load_4d(sV + HALF_BYTES, &tmv, bar(KV_FULL), 64, h, kv0, b);
+            const uint64_t keep = l2_policy_evict_last();
+            int par[2] = {-1, -1};
+            bool ok = true;
+            for (int i = 0; i < nq; ++i) {
+                const int s = i & 1;
+                const int use = (i >> 1) & 1;
+                ok = wait_thread(bar(QDO_EMPTY + s), use ^ 1, wc);
+                if (!ok) break;
+                const uint32_t fb = bar(QDO_FULL + s);
+                mbar_arrive_expect_tx(fb, 2 * TILE_BYTES);
+                tma_load_4d_hint(sQ + s * TILE_BYTES, &tmq, fb, 0, h, i * BM, b, keep);
+                tma_load_4d_hint(sQ + s * TILE_BYTES + HALF_BYTES, &tmq, fb, 64, h, i * BM, b, keep);
+                tma_load_4d_hint(sDO + s * TILE_BYTES, &tmdo, fb, 0, h, i * BM, b, keep);
+                tma_load_4d_hint(sDO + s * TILE_BYTES + HALF_BYTES, &tmdo, fb, 64, h, i * BM, b, keep);
+                par[s] = use;
+            }
+            if (!ok) {
+                drain_wait(bar(KV_FULL), 0, p.wait_budget_ns);
+                for (int s = 0; s < 2; ++s)
+                    if (par[s] >= 0) drain_wait(bar(QDO_FULL + s), par[s], p.wait_budget_ns);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------ MMA issuer --------------------------------
+        if (lane == 0) {
+            const uint32_t id_kk = make_idesc(1, 1, 1, 0, 0, BM, BM);   // both K-major
+            const uint32_t id_tb = make_idesc(1, 1, 1, 0, 1, BM, HD);   // A in TMEM, B MN-major
+            const uint32_t id_mm = make_idesc(1, 1, 1, 1, 1, HD, BM);   // both MN-major
+            bool ok = wait_thread(bar(KV_FULL), 0, wc);
+            for (int i = 0; i < nq && ok; ++i) {
+                const int s = i & 1;
+                ok = wait_thread(bar(QDO_FULL + s), (i >> 1) & 1, wc);
+                if (ok && i > 0) ok = wait_thread(bar(DQ_DRAINED), (i - 1) & 1, wc);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t q_s = sQ + s * TILE_BYTES, do_s = sDO + s * TILE_BYTES;
+                mma_kmajor(tmem + T_S, sK, q_s, id_kk, false);        // S^T = K Q^T
+                mma_commit(bar(S_FULL));
+                mma_kmajor(tmem + T_DP, sV, do_s, id_kk, false);      // dP^T = V dO^T
+                mma_commit(bar(DP_FULL));
+                ok = wait_thread(bar(P_READY), i & 1, wc);
+                if (!ok) break;
+                tc_fence_after();
+                mma_ts_bmn(tmem + T_DV, tmem + T_S, do_s, id_tb, i > 0);   // dV += P^T dO
+                mma_commit(bar(DV_DONE));
+                ok = wait_thread(bar(DS_READY), i & 1, wc);
+                if (!ok) break;
+                tc_fence_after();
+                mma_ts_bmn(tmem + T_DK, tmem + T_DP, q_s, id_tb, i > 0);   // dK += dS^T Q
+                mma_ss_mn(tmem + T_S, sK, do_s, id_mm);                    // dQ^T = K^T dS^T (dS^T in dO's buffer)
+                mma_commit(bar(DQ_FULL));
+                mma_commit(bar(QDO_EMPTY + s));
+            }
+            if (ok) mma_commit(bar(FINAL));
+            mma_commit(bar(DRAIN));
+            drain_wait(bar(DRAIN), 0, p.wait_budget_ns);
+        }
+    } else {
+        // -------------------- gradients warpgroup (thread = key row / d) -----------
+        const int j = threadIdx.x;                         // 0..127
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t tS = tmem + T_S + lane_off, tDP = tmem + T_DP + lane_off;
+        const int key = kv0 + j;
+        const bool key_ok = key < S;
+        const float c = p.scale_log2;
+        const size_t bh = static_cast<size_t>(b) * p.H + h;
+        // each warp keeps its own copy of the Q tile's lse / D (no cross-warp barrier needed)
+        float* s_lse = reinterpret_cast<float*>(smem + OFF_VEC + warp * VEC_BYTES);
+        float* s_del = s_lse + BM;
+        bool ok = true;
+        for (int i = 0; i < nq && ok; ++i) {
+            __syncwarp();                                    // previous tile's values no longer read
+#pragma unroll
+            for (int e = 0; e < BM / 32; ++e) {
+                const int col = e * 32 + lane;
+                const int qi = i * BM + col;
+                s_lse[col] = qi < S ? p.lse[bh * S + qi] * LOG2E : INFINITY;
+                s_del[col] = qi < S ? p.delta[bh * S + qi] : 0.f;
+            }
+            __syncwarp();
+
+            ok = wait_warp(bar(S_FULL), i & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            float pr[128];
+            {
+                uint32_t* sr = reinterpret_cast<uint32_t*>(pr);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q * 32]));
+                tmem_wait_ld();
+            }
+#pragma unroll
+            for (int e = 0; e < 128; ++e) pr[e] = key_ok ? ex2_approx(fmaf(pr[e], c, -s_lse[e])) : 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[half * 64 + 2 * e], pr[half * 64 + 2 * e + 1]);
+                tmem_st32(tS + half * 32, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(P_READY));
+
+            ok = wait_warp(bar(DP_FULL), i & 1, wc) && wait_warp(bar(DV_DONE), i & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            uint8_t* ds_row = smem + OFF_DO + (i & 1) * TILE_BYTES + j * 128;   // row j of both halves
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t dp[32];
+                tmem_ld32(tDP + q * 32, dp);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int c0 = q * 32 + 2 * e;
+                    const float d0 = pr[c0] * (__uint_as_float(dp[2 * e]) - s_del[c0]);
+                    const float d1 = pr[c0 + 1] * (__uint_as_float(dp[2 * e + 1]) - s_del[c0 + 1]);
+                    pk[e] = pack_bf16x2(d0, d1);
+                }
+                tmem_st16(tDP + q * 16, pk);
+                // dS^T row j, queries 32q..32q+31 -> 128-byte swizzled row of half q/2
+                uint8_t* half_row = ds_row + (q >> 1) * HALF_BYTES;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int chunk = ((q & 1) * 4 + ch) ^ (j & 7);
+                    *reinterpret_cast<uint4*>(half_row + chunk * 16) =
+                        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+                }
+            }
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(DS_READY));
+
+            ok = wait_warp(bar(DQ_FULL), i & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            // dQ^T: TMEM lane = d (this thread's j), column = query within the tile
+            float* dq_col = p.dq_acc + h * HD + j;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                tmem_ld32(tS + q * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int query = i * BM + q * 32 + e;
+                    if (query < S)
+                        atomicAdd(dq_col + (static_cast<size_t>(b) * S + query) * (static_cast<size_t>(p.H) * HD),
+                                  __uint_as_float(v[e]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(DQ_DRAINED));
+        }
+        if (ok) ok = wait_warp(bar(FINAL), 0, wc);
+        if (ok) {
+            tc_fence_after();
+            const size_t row = ((static_cast<size_t>(b) * S + key) * p.H + h) * HD;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t src = tmem + (which ? T_DK : T_DV) + lane_off;
+                const float mul = which ? p.scale : 1.f;
+                __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(which ? p.dk : p.dv) + row;
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t v[32];
+                    tmem_ld32(src + q * 32, v);
+                    tmem_wait_ld();
+                    uint4 pk[4];
+                    uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pw[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+                    if (key_ok) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + q * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) d4[e] = pk[e];
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// D_i = sum_d dO_id * O_id (fp32) for every (b, s, h) row, and dQ accumulator := 0.
+// 16 threads per row, 8 elements (16 bytes) each.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ dout,
+                                                       float* __restrict__ delta, float* __restrict__ dq_acc,
+                                                       long long rows, int S, int H) {
+    const long long total = rows * 16;
+    const int lane = threadIdx.x & 31;
+    const long long warp0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x - lane;
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long t0 = warp0; t0 < total; t0 += stride) {        // warp-uniform trip count
+        const long long t = t0 + lane;
+        const bool valid = t < total;
+        const long long r = t >> 4;               // row index over [B, S, H]
+        const int part = static_cast<int>(t & 15);
+        float acc = 0.f;
+        if (valid) {
+            const uint4 ov = *reinterpret_cast<const uint4*>(o + r * HD + part * 8);
+            const uint4 dv = *reinterpret_cast<const uint4*>(dout + r * HD + part * 8);
+            const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+            const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 a = __bfloat1622float2(o2[e]);
+                const float2 c = __bfloat1622float2(d2[e]);
+                acc = fmaf(a.x, c.x, acc);
+                acc = fmaf(a.y, c.y, acc);
+            }
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (valid) {
+            float4* z = reinterpret_cast<float4*>(dq_acc + r * HD + part * 8);
+            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (part == 0) {
+                const long long h = r % H;
+                const long long bs = r / H;
+                const long long s = bs % S;
+                const long long b = bs / S;
+                delta[(b * H + h) * S + s] = acc;
+            }
+        }
+    }
+}
+
+// dQ = bf16(acc * scale), 8 elements per thread.
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
+                                                     long long n8, float scale) {
+    const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long t = tid; t < n8; t += stride) {
+        const float4 a = reinterpret_cast<const float4*>(acc)[2 * t];
+        const float4 c = reinterpret_cast<const float4*>(acc)[2 * t + 1];
+        uint4 out;
+        out.x = pack_bf16x2(a.x * scale, a.y * scale);
+        out.y = pack_bf16x2(a.z * scale, a.w * scale);
+        out.z = pack_bf16x2(c.x * scale, c.y * scale);
+        out.w = pack_bf16x2(c.z * scale, c.w * scale);
+        reinterpret_cast<uint4*>(dq)[t] = out;
+    }
+}
+
+}  // namespace bwd
+
+int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+               const BwdParams& p, const void* o, const void* dout, void* dq, cudaStream_t stream) {
+    const long long rows = static_cast<long long>(p.B) * p.S * p.H;
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int ew_blocks = sms * 8;     // grid-stride elementwise kernels: 8 blocks of 256 per SM
+    bwd::bwd_prep_kernel<<<ew_blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                        static_cast<const __nv_bfloat16*>(dout), p.delta, p.dq_acc,
+                                                        rows, p.S, p.H);
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    if (configure_smem(reinterpret_cast<const void*>(bwd::bwd_main_kernel), bwd::SMEM_BYTES) != 0) return -1;
+    const dim3 grid((p.S + bwd::BM - 1) / bwd::BM, p.H, p.B);
+    bwd::bwd_main_kernel<<<grid, bwd::NTHREADS, bwd::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    bwd::bwd_dq_kernel<<<ew_blocks, 256, 0, stream>>>(p.dq_acc, static_cast<__nv_bfloat16*>(dq), rows * 16,
+                                                      p.scale);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace wan

@@ -18,6 +18,19 @@ struct FwdParams {
     int* status;                // device status word (see wan_attn_sync_status)
 };
 
+struct BwdParams {
+    const float* lse;           // fp32 [B, H, S] from the forward (natural log)
+    float* delta;               // workspace fp32 [B, H, S]: rowsum(dO * O)
+    float* dq_acc;              // workspace fp32 [B, S, H, 128]: unscaled dS K
+    void* dk;                   // bf16 [B, S, H, 128]
+    void* dv;                   // bf16 [B, S, H, 128]
+    int B, S, H;
+    float scale;                // 1 / sqrt(D)
+    float scale_log2;           // scale * log2(e)
+    unsigned long long wait_budget_ns;
+    int* status;
+};
+
 // Device address of the status word on the current device (nullptr on failure).
 int* device_status_word();
 unsigned long long wait_budget_ns();
@@ -27,5 +40,8 @@ int configure_smem(const void* kernel, int bytes);
 
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                cudaStream_t stream);
+
+int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+               const BwdParams& p, const void* o, const void* dout, void* dq, cudaStream_t stream);
 
 }  // namespace wan

@@ -21,6 +21,8 @@ STATUS = {0: "WAN_ATTN_OK", 1: "WAN_ATTN_ERR_INVALID_ARG", 2: "WAN_ATTN_ERR_UNSU
 _P, _I, _Z, _U64, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_void_p
 SIGNATURES = [
     ("wan_attn_fwd", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P]),
+    ("wan_attn_bwd_workspace_size", _Z, [_I, _I, _I, _I]),
+    ("wan_attn_bwd", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]),
     ("wan_attn_sync_status", _I, [_P]),
     ("wan_attn_status_string", ctypes.c_char_p, [_I]),
     ("wan_attn_set_wait_budget_ns", _U64, [_U64]),
@@ -94,6 +96,34 @@ def fwd(q, k, v, o=None, lse=None, stream=None):
     _check("wan_attn_fwd", lib().wan_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                               lse.data_ptr(), B, S, H, D, _stream_ptr(stream)))
     return o, lse
+
+
+def bwd_workspace_size(B, S, H, D=128) -> int:
+    return lib().wan_attn_bwd_workspace_size(B, S, H, D)
+
+
+def bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of sum(O * dO) through ``wan_attn_bwd``; outputs/workspace allocated if not given."""
+    import torch
+    _check_bshd("q", q)
+    B, S, H, D = q.shape
+    for name, t in (("k", k), ("v", v), ("o", o), ("do", do)):
+        _check_bshd(name, t, q.shape)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, S) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, S] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_bshd(name, t, q.shape)
+    need = bwd_workspace_size(B, S, H, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check("wan_attn_bwd", lib().wan_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                              dv.data_ptr(), B, S, H, D, workspace.data_ptr(),
+                                              workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
+    return dq, dk, dv
 
 
 def sync_status(stream=None) -> int:
