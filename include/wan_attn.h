@@ -95,6 +95,36 @@ WAN_ATTN_API int wan_attn_bwd(const void* q, const void* k, const void* v, const
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Size of the library's own backward workspace used by wan_attn_bwd_noalloc:
+ * 32 MiB, held on every GPU that loads the library until the process exits.
+ * It fits B*S*H <= 65027 (token, head) rows, e.g. B=1, S=2048, H=24.
+ */
+#define WAN_ATTN_NOALLOC_WORKSPACE_BYTES (32u << 20)
+
+/*
+ * The backward of wan_attn_bwd without a caller-supplied workspace: no
+ * counterpart in the pages; it serves callers that cannot allocate device
+ * memory (a plugin whose host application owns all device memory and hands
+ * out no allocator, or a server that forbids cudaMalloc after start-up since
+ * it can synchronise the device and fragment memory).  Arguments, layouts,
+ * results and errors are those of wan_attn_bwd, minus the workspace, which is
+ * a fixed WAN_ATTN_NOALLOC_WORKSPACE_BYTES device array inside the library.
+ *   - Sizes whose wan_attn_bwd_workspace_size(B, S, H, D) exceeds that array
+ *     return WAN_ATTN_ERR_WORKSPACE and enqueue nothing.
+ *   - The call allocates and frees nothing.  Its first call on a device looks
+ *     up the array's device address (cudaGetSymbolAddress) with that device
+ *     current; make that first call before any stream capture.
+ *   - Every call on a device shares the one array.  Calls whose kernels
+ *     overlap on the GPU (other streams, other host threads) race on it:
+ *     order them on one stream or with events.  Each call clears what must
+ *     start at zero, so a finished earlier call leaves nothing behind that
+ *     matters.
+ */
+WAN_ATTN_API int wan_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                      const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                                      int B, int S, int H, int D, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word:
  * WAN_ATTN_OK, WAN_ATTN_ERR_TIMEOUT (a kernel's bounded wait ran out), or
  * WAN_ATTN_ERR_CUDA if the synchronisation itself failed.

@@ -23,6 +23,7 @@ SIGNATURES = [
     ("wan_attn_fwd", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P]),
     ("wan_attn_bwd_workspace_size", _Z, [_I, _I, _I, _I]),
     ("wan_attn_bwd", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]),
+    ("wan_attn_bwd_noalloc", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _P]),
     ("wan_attn_sync_status", _I, [_P]),
     ("wan_attn_status_string", ctypes.c_char_p, [_I]),
     ("wan_attn_set_wait_budget_ns", _U64, [_U64]),
