@@ -31,6 +31,10 @@ import synth  # noqa: E402
 
 METRIC = "attention TFLOP/s (4*B*H*S^2*D fwd)"
 
+# DRAM bytes (read + write) of one launch of the dominant kernel from an ncu
+# capture (profiles/), per workload; None where the kernel changed since.
+TRAFFIC = {"wan14b_720p": 3.335e9}
+
 
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -150,6 +154,80 @@ def run_reference(args, w):
     return 0
 
 
+class Path:
+    """The calls one bench step makes for a workload, with their buffers.
+
+    fwd workloads: one wan_attn_fwd; the training workload: wan_attn_fwd then
+    wan_attn_bwd; the 8-bit workload: one wan_attn_fwd_q8 (quantise + attend).
+    """
+
+    def __init__(self, wa, w, dev, x):
+        import torch
+        self.wa, self.w = wa, w
+        shape = (w.B, w.S, w.H, w.D)
+
+        def pinned(bits):
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+        names = ["q", "k", "v"] + (["do"] if w.backward else [])
+        self.host_in = [pinned(x[n]) for n in names]
+        self.dev_in = [t.to(dev) for t in self.host_in]
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty(shape, **bf)
+        self.lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+        self.outs = [self.o, self.lse]
+        self.ws = None
+        if w.backward:
+            self.grads = [torch.empty(shape, **bf) for _ in range(3)]
+            self.ws = torch.empty(wa.bwd_workspace_size(w.B, w.S, w.H, w.D), dtype=torch.uint8, device=dev)
+            self.outs = self.outs + self.grads
+            self.flop = 3.5 * w.fwd_flop                   # forward + 2.5x forward for the backward
+            self.dominant_flop = 2.5 * w.fwd_flop
+            self.kernel = "wan::bwd::bwd_main_kernel (timed with its prep and dQ kernels: one wan_attn_bwd call)"
+            self.launches_per_step = 4
+            self.peak_key, self.dtype = "bf16", "bf16"
+        elif w.q8:
+            self.ws = torch.empty(wa.fwd_q8_workspace_size(w.B, w.S, w.H, w.D), dtype=torch.uint8, device=dev)
+            self.flop = w.fwd_flop
+            self.dominant_flop = w.fwd_flop
+            self.kernel = "wan::q8::q8_attn_kernel (timed with its quantise kernel: one wan_attn_fwd_q8 call)"
+            self.launches_per_step = 2
+            self.peak_key, self.dtype = "fp8", "int8/e4m3"
+        else:
+            self.flop = w.fwd_flop
+            self.dominant_flop = w.fwd_flop
+            self.kernel = "wan::fwd::attn_fwd_kernel"
+            self.launches_per_step = 1
+            self.peak_key, self.dtype = "bf16", "bf16"
+        self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.host_in)
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.host_out)
+
+    def step(self, dom_events=None):
+        wa, (q, k, v) = self.wa, self.dev_in[:3]
+        if self.w.backward:
+            wa.fwd(q, k, v, self.o, self.lse)
+            if dom_events:
+                dom_events[0].record()
+            wa.bwd(q, k, v, self.o, self.dev_in[3], self.lse, *self.grads, workspace=self.ws)
+        else:
+            if dom_events:
+                dom_events[0].record()
+            if self.w.q8:
+                wa.fwd_q8(q, k, v, self.o, self.lse, workspace=self.ws)
+            else:
+                wa.fwd(q, k, v, self.o, self.lse)
+        if dom_events:
+            dom_events[1].record()
+
+    def e2e_step(self):
+        for d, h in zip(self.dev_in, self.host_in):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        for h, d in zip(self.host_out, self.outs):
+            h.copy_(d, non_blocking=True)
+
+
 def run_ours(args, w):
     import torch
     import video_dit_full_b200 as wa
@@ -158,39 +236,35 @@ def run_ours(args, w):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dist = None
+    torch.cuda.set_device(local)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     wa.lib()
 
     # each rank gets its own seeded problem (seed = rank): weak scaling
     x = synth.make_inputs(w, seed=rank)
-    shape = (w.B, w.S, w.H, w.D)
-
-    def host_pinned(bits):
-        t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
-        return t.pin_memory()
-
-    hq, hk, hv = (host_pinned(x[n]) for n in "qkv")
-    q, k, v = (t.to(dev) for t in (hq, hk, hv))
-    o = torch.empty(shape, dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+    path = Path(wa, w, dev, x)
     stream = torch.cuda.current_stream(dev)
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
+    def max_over_ranks(ms):
+        if dist is None:
+            return ms
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
     # ------------------------ device-resident timing ------------------------
     for _ in range(args.warmup):
-        wa.fwd(q, k, v, o, lse)
-    wa.check_status()
+        path.step()
+    status = wa.sync_status()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     sampler = ClockSampler(nvsmi_id(dev, local))
     barrier()
@@ -200,75 +274,60 @@ def run_ours(args, w):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for s in range(args.steps):
-        ev[s][0].record(stream)
-        wa.fwd(q, k, v, o, lse)
-        ev[s][1].record(stream)
+        path.step(ev[s])
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     barrier()
-    status = wa.sync_status()
-    total_ms = t_start.elapsed_time(t_end)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    status = status or wa.sync_status()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    dom_ms = [a.elapsed_time(b) for a, b in ev]
     ms_per_step = total_ms / args.steps
-    value = world * w.fwd_flop * args.steps / (total_ms * 1e-3) / 1e12
+    value = world * path.flop * args.steps / (total_ms * 1e-3) / 1e12
 
     # ------------------- end to end through host buffers ---------------------
-    ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
-    hl = torch.empty((w.B, w.H, w.S), dtype=torch.float32).pin_memory()
     e2e_steps = max(1, min(args.steps, 5))
-
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        wa.fwd(q, k, v, o, lse)
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
-
-    e2e_step()
+    path.e2e_step()
     torch.cuda.synchronize(dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        e2e_step()
+        path.e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * w.fwd_flop * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = world * path.flop * e2e_steps / (e2e_ms * 1e-3) / 1e12
     status = status or wa.sync_status()
 
     if rank == 0:
         peaks = load_peaks()
-        mean_launch_ms = sum(launch_ms) / len(launch_ms)
-        achieved = w.fwd_flop / (mean_launch_ms * 1e-3) / 1e12
+        mean_ms = sum(dom_ms) / len(dom_ms)
+        achieved = path.dominant_flop / (mean_ms * 1e-3) / 1e12
+        if path.peak_key == "fp8":
+            peak = 2.0 * peaks["bf16"]
+            peak_src = f"{peaks['source']} bf16 dense burst x 2 (nominal fp8/int8 : bf16 ratio)"
+            sustained = 2.0 * peaks["bf16_sustained"]
+        else:
+            peak, sustained = peaks["bf16"], peaks["bf16_sustained"]
+            peak_src = f"{peaks['source']} bf16 dense (burst)"
+        in_gb = sum(t.numel() * t.element_size() for t in path.dev_in) / 1e9
         line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC if not w.backward else "attention TFLOP/s (fwd 4*B*H*S^2*D + bwd 2.5x fwd)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": path.dtype, "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "S": w.S, "H": w.H, "D": w.D,
-                       "fwd_flop_per_step": w.fwd_flop, "parallelism": f"replicas{world}",
-                       "l2": "inputs (Q, K, V: %.2f GB) exceed the 126 MB L2; no flush" % (3 * w.B * w.S * w.H * w.D * 2 / 1e9)},
-            "gpu_launches": args.steps,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s",
-                         "frac": achieved / peaks["bf16"], "traffic": None,
-                         "peak_source": f"{peaks['source']} bf16 dense (burst)",
-                         "frac_of_sustained": achieved / peaks["bf16_sustained"],
-                         "kernel": "wan::fwd::attn_fwd_kernel",
-                         "launch_ms": {"mean": mean_launch_ms, "min": min(launch_ms), "max": max(launch_ms)}},
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": 3 * w.B * w.S * w.H * w.D * 2,
-                    "d2h_bytes_per_step": w.B * w.S * w.H * w.D * 2 + w.B * w.H * w.S * 4,
-                    "steps": e2e_steps},
+                       "flop_per_step": path.flop, "parallelism": f"replicas{world}",
+                       "l2": "inputs (%.2f GB) exceed the 126 MB L2; no flush" % in_gb},
+            "gpu_launches": args.steps * path.launches_per_step,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": TRAFFIC.get(w.name),
+                         "peak_source": peak_src, "frac_of_sustained": achieved / sustained,
+                         "kernel": path.kernel,
+                         "launch_ms": {"mean": mean_ms, "min": min(dom_ms), "max": max(dom_ms)}},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": path.h2d_bytes,
+                    "d2h_bytes_per_step": path.d2h_bytes, "steps": e2e_steps},
             "clocks": clocks,
             "device_status": status,
         }

@@ -95,6 +95,40 @@ WAN_ATTN_API int wan_attn_bwd(const void* q, const void* k, const void* v, const
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Bytes of device workspace wan_attn_fwd_q8 needs: the quantised copies and
+ * their scales, each part starting on a 256-byte boundary, in this order:
+ *   int8 Q8 [B, H, S, D], int8 K8 [B, H, S, D], e4m3 V8 [B, H, S, D],
+ *   fp32 sQ, sK, sV [B, H, ceil(S/64)].
+ * Returns 0 if the sizes are invalid.
+ */
+WAN_ATTN_API size_t wan_attn_fwd_q8_workspace_size(int B, int S, int H, int D);
+
+/*
+ * 8-bit forward: the pages' 8-bit FlashAttention ("Wan 2.1 ..." paper-podcast
+ * summary, section "干预与形式化": mixed int8/FP8 with FP32 accumulation
+ * across blocks; kwkr.cn Wan explainer, section 4.2).  Read as:
+ *   - per (b, h, 64-token block): sQ = absmax(Q)/127, sK = absmax(K)/127,
+ *     sV = absmax(V)/448 (fp32; 1 for an all-zero block); codes
+ *     Q8 = clamp(rint(q / sQ), -127, 127), K8 likewise, V8 = e4m3(v / sV),
+ *     each division IEEE fp32, rounding to nearest even, e4m3 saturating;
+ *   - scores S = (Q8 . K8) sQ sK / sqrt(D) from int32 tensor-core sums;
+ *   - P8 = e4m3(448 * exp(S - running max)); each 64-key block's P8 V8
+ *     product is taken out of the tensor core in fp32 and added to O with
+ *     that block's sV; the row sum uses the unquantised exponentials.
+ *   q, k, v : in,  bf16 [B, S, H, D]
+ *   o       : out, bf16 [B, S, H, D]
+ *   lse     : out, fp32 [B, H, S], natural log, of the dequantised scores
+ *   workspace, workspace_bytes : caller-owned device memory, 256-byte aligned,
+ *             at least wan_attn_fwd_q8_workspace_size bytes (else
+ *             WAN_ATTN_ERR_WORKSPACE); on return it holds the quantised
+ *             tensors and scales in the layout above.
+ * Other conventions as wan_attn_fwd.
+ */
+WAN_ATTN_API int wan_attn_fwd_q8(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int B, int S, int H, int D, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
  * Size of the library's own backward workspace used by wan_attn_bwd_noalloc:
  * 32 MiB, held on every GPU that loads the library until the process exits.
  * It fits B*S*H <= 65027 (token, head) rows, e.g. B=1, S=2048, H=24.

@@ -90,3 +90,16 @@ def test_bwd_host_side_validation_without_gpu(built):
     assert lib.wan_attn_bwd(*args(ws=ctypes.c_void_p(0x100000 + 9 * 0x1000000 + 16))) == WORKSPACE
     assert lib.wan_attn_bwd(*args(dq=q)) == INVALID                 # output aliases an input
     assert lib.wan_attn_bwd(*args(dk=dv)) == INVALID                # two outputs alias
+
+
+def test_q8_host_side_validation_without_gpu(built):
+    from video_dit_full_b200 import wan_attn
+    lib = wan_attn.lib()
+    q, k, v, o, lse, ws = (ctypes.c_void_p(0x100000 + i * 0x10000000) for i in range(6))
+    need = lib.wan_attn_fwd_q8_workspace_size(1, 130, 2, 128)
+    assert need == 3 * 33280 + 3 * 256      # 3 x align256(130*2*128) + 3 x align256(2*3*4)
+    assert lib.wan_attn_fwd_q8_workspace_size(1, 130, 2, 100) == 0
+    assert lib.wan_attn_fwd_q8(q, k, v, o, lse, 1, 130, 2, 128, None, need, None) == 5
+    assert lib.wan_attn_fwd_q8(q, k, v, o, lse, 1, 130, 2, 128, ws, need - 1, None) == 5
+    assert lib.wan_attn_fwd_q8(q, k, v, q, lse, 1, 130, 2, 128, ws, need, None) == 1
+    assert lib.wan_attn_fwd_q8(q, k, v, o, lse, 1, 130, 2, 120, ws, need, None) == 2

@@ -3,5 +3,6 @@
 The computation lives in ``libwan_attn.so`` (hand-written CUDA for sm_100a,
 C ABI in ``include/wan_attn.h``); ``wan_attn`` is its ctypes binding.
 """
-from .wan_attn import (WanAttnError, bwd, bwd_workspace_size, check_status, fwd, lib, selftest_wait_timeout,  # noqa: F401
+from .wan_attn import (WanAttnError, bwd, bwd_workspace_size, check_status, fwd, fwd_q8, fwd_q8_workspace_size, lib,
+                       q8_workspace_views, selftest_wait_timeout,  # noqa: F401
                        set_wait_budget_ns, sync_status)

@@ -61,6 +61,20 @@ bool make_bshd_map(CUtensorMap* m, const void* base, int B, int S, int H, int D,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map over an 8-bit [B*H, S, 128] tensor viewed as 3-D (128, S, B*H), box (128, 128, 1),
+// 128-byte swizzle (one 128-byte row per token), tokens past S read as zero.
+bool make_bh_s_d8_map(CUtensorMap* m, const void* base, int BH, int S) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {128, (cuuint64_t)S, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)S * 128};
+    const cuuint32_t box[3] = {128, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Range {
     uintptr_t lo, hi;
 };
@@ -204,6 +218,70 @@ int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
     if (!p.status) return WAN_ATTN_ERR_CUDA;
     return launch_bwd(tq, tk, tv, tdo, p, o, dO, dq, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
                                                                                           : WAN_ATTN_ERR_CUDA;
+}
+
+size_t wan_attn_fwd_q8_workspace_size(int B, int S, int H, int D) {
+    if (check_shape(B, S, H, D) != WAN_ATTN_OK) return 0;
+    const size_t n = size_t(B) * S * H * D;
+    const size_t nblk = (size_t(S) + 63) / 64;
+    return 3 * align256(n) + 3 * align256(size_t(B) * H * nblk * 4);
+}
+
+int wan_attn_fwd_q8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S, int H, int D,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !o || !lse) return WAN_ATTN_ERR_INVALID_ARG;
+    const int st = check_shape(B, S, H, D);
+    if (st != WAN_ATTN_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return WAN_ATTN_ERR_INVALID_ARG;
+    const size_t need = wan_attn_fwd_q8_workspace_size(B, S, H, D);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return WAN_ATTN_ERR_WORKSPACE;
+    const size_t n = size_t(B) * S * H * D;
+    const Range ins[] = {range_of(q, n * 2), range_of(k, n * 2), range_of(v, n * 2)};
+    const Range outs[] = {range_of(o, n * 2), range_of(lse, size_t(B) * H * S * 4), range_of(workspace, need)};
+    for (size_t a = 0; a < 3; ++a) {
+        for (const Range& in : ins)
+            if (overlaps(outs[a], in)) return WAN_ATTN_ERR_INVALID_ARG;
+        for (size_t c = a + 1; c < 3; ++c)
+            if (overlaps(outs[a], outs[c])) return WAN_ATTN_ERR_INVALID_ARG;
+    }
+    const int nblk = (S + 63) / 64;
+    char* ws = static_cast<char*>(workspace);
+    const size_t code_bytes = align256(n), scale_bytes = align256(size_t(B) * H * nblk * 4);
+    Q8QuantParams qp;
+    qp.q = static_cast<const __nv_bfloat16*>(q);
+    qp.k = static_cast<const __nv_bfloat16*>(k);
+    qp.v = static_cast<const __nv_bfloat16*>(v);
+    qp.q8 = reinterpret_cast<int8_t*>(ws);
+    qp.k8 = reinterpret_cast<int8_t*>(ws + code_bytes);
+    qp.v8 = reinterpret_cast<uint8_t*>(ws + 2 * code_bytes);
+    qp.sq = reinterpret_cast<float*>(ws + 3 * code_bytes);
+    qp.sk = reinterpret_cast<float*>(ws + 3 * code_bytes + scale_bytes);
+    qp.sv = reinterpret_cast<float*>(ws + 3 * code_bytes + 2 * scale_bytes);
+    qp.B = B;
+    qp.S = S;
+    qp.H = H;
+    qp.nblk = nblk;
+    CUtensorMap tq, tk, tv;
+    if (!make_bh_s_d8_map(&tq, qp.q8, B * H, S) || !make_bh_s_d8_map(&tk, qp.k8, B * H, S) ||
+        !make_bh_s_d8_map(&tv, qp.v8, B * H, S))
+        return WAN_ATTN_ERR_CUDA;
+    Q8AttnParams p;
+    p.o = o;
+    p.lse = lse;
+    p.sq = qp.sq;
+    p.sk = qp.sk;
+    p.sv = qp.sv;
+    p.B = B;
+    p.S = S;
+    p.H = H;
+    p.nblk = nblk;
+    p.scale_log2 = static_cast<float>((1.0 / std::sqrt(double(D))) * 1.4426950408889634);
+    p.wait_budget_ns = wait_budget_ns();
+    p.status = device_status_word();
+    if (!p.status) return WAN_ATTN_ERR_CUDA;
+    return launch_q8(qp, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
 }
 
 int wan_attn_sync_status(void* stream) {

@@ -31,6 +31,24 @@ struct BwdParams {
     int* status;
 };
 
+struct Q8QuantParams {
+    const __nv_bfloat16 *q, *k, *v;   // bf16 [B, S, H, 128]
+    int8_t *q8, *k8;                  // int8 [B, H, S, 128]
+    uint8_t* v8;                      // e4m3 [B, H, S, 128]
+    float *sq, *sk, *sv;              // fp32 [B, H, nblk]
+    int B, S, H, nblk;
+};
+
+struct Q8AttnParams {
+    void* o;                          // bf16 [B, S, H, 128]
+    float* lse;                       // fp32 [B, H, S]
+    const float *sq, *sk, *sv;        // fp32 [B, H, nblk]
+    int B, S, H, nblk;
+    float scale_log2;
+    unsigned long long wait_budget_ns;
+    int* status;
+};
+
 // Device address of the status word on the current device (nullptr on failure).
 int* device_status_word();
 unsigned long long wait_budget_ns();
@@ -43,5 +61,8 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
 
 int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                const BwdParams& p, const void* o, const void* dout, void* dq, cudaStream_t stream);
+
+int launch_q8(const Q8QuantParams& qp, const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv8,
+              const Q8AttnParams& p, cudaStream_t stream);
 
 }  // namespace wan

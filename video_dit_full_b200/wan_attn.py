@@ -23,6 +23,8 @@ SIGNATURES = [
     ("wan_attn_fwd", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P]),
     ("wan_attn_bwd_workspace_size", _Z, [_I, _I, _I, _I]),
     ("wan_attn_bwd", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]),
+    ("wan_attn_fwd_q8_workspace_size", _Z, [_I, _I, _I, _I]),
+    ("wan_attn_fwd_q8", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P, _Z, _P]),
     ("wan_attn_bwd_noalloc", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _P]),
     ("wan_attn_sync_status", _I, [_P]),
     ("wan_attn_status_string", ctypes.c_char_p, [_I]),
@@ -125,6 +127,45 @@ def bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None, stream=N
                                               dv.data_ptr(), B, S, H, D, workspace.data_ptr(),
                                               workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
     return dq, dk, dv
+
+
+def fwd_q8_workspace_size(B, S, H, D=128) -> int:
+    return lib().wan_attn_fwd_q8_workspace_size(B, S, H, D)
+
+
+def fwd_q8(q, k, v, o=None, lse=None, workspace=None, stream=None):
+    """O, LSE of the 8-bit forward through ``wan_attn_fwd_q8``; returns (o, lse, workspace)."""
+    import torch
+    _check_bshd("q", q)
+    B, S, H, D = q.shape
+    _check_bshd("k", k, q.shape)
+    _check_bshd("v", v, q.shape)
+    o = torch.empty_like(q) if o is None else o
+    _check_bshd("o", o, q.shape)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, S) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, S] tensor")
+    if workspace is None:
+        workspace = torch.empty(fwd_q8_workspace_size(B, S, H, D), dtype=torch.uint8, device=q.device)
+    _check("wan_attn_fwd_q8", lib().wan_attn_fwd_q8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                                    lse.data_ptr(), B, S, H, D, workspace.data_ptr(),
+                                                    workspace.numel() * workspace.element_size(),
+                                                    _stream_ptr(stream)))
+    return o, lse, workspace
+
+
+def q8_workspace_views(workspace, B, S, H, D=128):
+    """Views of a wan_attn_fwd_q8 workspace: (q8, k8, v8 as uint8 [B, H, S, D], sq, sk, sv fp32 [B, H, nblk])."""
+    import torch
+    n = B * S * H * D
+    nblk = (S + 63) // 64
+    a = lambda x: (x + 255) // 256 * 256
+    cb, sb = a(n), a(B * H * nblk * 4)
+    codes = [workspace[i * cb:i * cb + n].view(B, H, S, D) for i in range(3)]
+    scales = [workspace[3 * cb + i * sb:3 * cb + i * sb + B * H * nblk * 4].view(torch.float32).view(B, H, nblk)
+              for i in range(3)]
+    return (*codes, *scales)
 
 
 def sync_status(stream=None) -> int:
