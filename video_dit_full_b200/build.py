@@ -2,6 +2,8 @@
 
     python -m video_dit_full_b200.build [--verbose]
 
+Extra nvcc flags (tuning macros such as -DWAN_FWD_POLY_PAIRS=3) can be passed
+in the WAN_ATTN_NVCC_FLAGS environment variable; use --force after changing it.
 Each ``csrc/*.cu`` is compiled to an object under ``_build/`` (skipped when
 up to date) and the objects are linked into ``video_dit_full_b200/libwan_attn.so``.
 """
@@ -43,7 +45,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         if (not force and os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(src)
                 and os.path.getmtime(obj) >= newest_header):
             continue
-        cmd = [nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
+        cmd = [nvcc(), *ARCH, *FLAGS, *os.environ.get("WAN_ATTN_NVCC_FLAGS", "").split(), "-c", src, "-o", obj]
         if verbose:
             cmd += ["-Xptxas", "-v"]
         print(" ".join(cmd), file=sys.stderr)

@@ -317,6 +317,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// 2^x on the FMA and integer pipes instead of the MUFU: x = n + f with n the
+// nearest integer (adding 1.5 * 2^23 rounds x into the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial fitted for minimax relative
+// error by video_dit_full_b200/fit_exp2_poly.py (max relative error 7.5e-5,
+// far below bf16's 2^-9); 2^n is added to the exponent field.  x is clamped to
+// -125 so the result stays a normal float (an input of -inf gives 2^-125.5).
+__device__ __forceinline__ float exp2_poly3(float x) {
+    x = fmaxf(x, -125.f);
+    const float j = x + 12582912.f;
+    const float f = x - (j - 12582912.f);
+    float p = fmaf(0.05517149344086647f, f, 0.24261093139648438f);
+    p = fmaf(p, f, 0.6932609677314758f);
+    p = fmaf(p, f, 0.9999280571937561f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
+}
+
 // Two floats -> packed bf16x2, round to nearest even; `lo` lands in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
