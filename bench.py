@@ -350,8 +350,13 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=128, help="query rows per head timed for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="query rows per head per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--S", type=int, default=None, help="override the token count (small profiling cases)")
+    ap.add_argument("--H", type=int, default=None, help="override the head count (small profiling cases)")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.S or args.H:
+        import dataclasses
+        w = dataclasses.replace(w, S=args.S or w.S, H=args.H or w.H, name=f"{w.name}@S{args.S or w.S}H{args.H or w.H}")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

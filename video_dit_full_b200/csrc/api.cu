@@ -7,7 +7,7 @@
 #include <set>
 #include <utility>
 
-#include "../../include/wan_attn.h"
+#include "wan_attn.h"
 #include "sm100_ptx.cuh"
 #include "wan_attn_internal.h"
 
@@ -72,6 +72,20 @@ bool make_bh_s_d8_map(CUtensorMap* m, const void* base, int BH, int S) {
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor map over the fp32 dQ accumulator [B, S, H, 128] as 4-D (128, H, S, B), box
+// (128, 1, 128, 1) without swizzle: the backward adds [128 query][128 d] tiles into it.
+bool make_dq_acc_map(CUtensorMap* m, void* base, int B, int S, int H) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {128 * 4, (cuuint64_t)H * 128 * 4, (cuuint64_t)S * H * 128 * 4};
+    const cuuint32_t box[4] = {128, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -198,9 +212,10 @@ int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
             if (overlaps(outs[a], outs[c])) return WAN_ATTN_ERR_INVALID_ARG;
     }
 
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, tdq;
     if (!make_bshd_map(&tq, q, B, S, H, D, 128) || !make_bshd_map(&tk, k, B, S, H, D, 128) ||
-        !make_bshd_map(&tv, v, B, S, H, D, 128) || !make_bshd_map(&tdo, dO, B, S, H, D, 128))
+        !make_bshd_map(&tv, v, B, S, H, D, 128) || !make_bshd_map(&tdo, dO, B, S, H, D, 128) ||
+        !make_dq_acc_map(&tdq, workspace, B, S, H))
         return WAN_ATTN_ERR_CUDA;
     BwdParams p;
     p.lse = lse;
@@ -216,7 +231,7 @@ int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
     p.wait_budget_ns = wait_budget_ns();
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
-    return launch_bwd(tq, tk, tv, tdo, p, o, dO, dq, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+    return launch_bwd(tq, tk, tv, tdo, tdq, p, o, dO, dq, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
                                                                                           : WAN_ATTN_ERR_CUDA;
 }
 

@@ -15,7 +15,8 @@
 //                 dV += P^T dO_i                            (A = P^T in TMEM)
 //                 dS^T = P^T (dP^T - D_i)  -> TMEM and smem (into dO_i's buffer)
 //                 dK += dS^T Q_i                            (A = dS^T in TMEM)
-//                 dQ_i^T = K^T dS^T  -> TMEM -> fp32 red.add into the accumulator
+//                 dQ_i^T = K^T dS^T  -> TMEM -> shared (fp32) -> TMA reduce-add into
+//                                       the accumulator (a dedicated reducer warp)
 //               P is recomputed from the forward's LSE; nothing of size S x S is stored.
 //   bwd_dq      dQ = bf16(accumulator / sqrt(D)).
 #include <cuda.h>
@@ -33,18 +34,20 @@ constexpr int HALF_BYTES = TILE_BYTES / 2;
 
 constexpr int OFF_K = 0;
 constexpr int OFF_V = OFF_K + TILE_BYTES;
-constexpr int OFF_Q = OFF_V + TILE_BYTES;          // 2 stages
-constexpr int OFF_DO = OFF_Q + 2 * TILE_BYTES;     // 2 stages (dS^T reuses the stage after dV)
-constexpr int OFF_VEC = OFF_DO + 2 * TILE_BYTES;   // per warp: 128 fp32 lse*log2(e), 128 fp32 D_i
+// Two stages of [Q_i | dO_i] (64 KB each).  Within a tile, dS^T overwrites dO_i once dV is done;
+// after the dK and dQ MMAs the whole stage holds the fp32 dQ^T tile [query][d] for the TMA reduce.
+constexpr int OFF_STAGE = OFF_V + TILE_BYTES;
+constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+constexpr int OFF_VEC = OFF_STAGE + 2 * STAGE_BYTES;   // per warp: 128 fp32 lse*log2(e), 128 fp32 D_i
 constexpr int VEC_BYTES = 2 * BM * 4;
 constexpr int OFF_BAR = OFF_VEC + 4 * VEC_BYTES;
 enum Bar { KV_FULL = 0, QDO_FULL = 1, QDO_EMPTY = 3, S_FULL = 5, DP_FULL = 6, P_READY = 7, DV_DONE = 8,
-           DS_READY = 9, DQ_FULL = 10, DQ_DRAINED = 11, FINAL = 12, DRAIN = 13, NBARS = 14 };
+           DS_READY = 9, DQ_FULL = 10, DQ_DRAINED = 11, FINAL = 12, DRAIN = 13, STAGED = 14, NBARS = 15 };
 constexpr int OFF_TMEM_SLOT = OFF_BAR + NBARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
 constexpr int SMEM_USED = OFF_ABORT + 8;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
-constexpr int NTHREADS = 192;            // warps 0-3 softmax/gradients, 4 TMA, 5 MMA
+constexpr int NTHREADS = 224;            // warps 0-3 gradients, 4 TMA, 5 MMA, 6 dQ reducer
 constexpr uint32_t TMEM_COLS = 512;      // S^T | dP^T | dV | dK
 constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -91,7 +94,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 __global__ void __launch_bounds__(NTHREADS, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
-                const BwdParams p) {
+                const __grid_constant__ CUtensorMap tmdq, const BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -104,7 +107,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     const int S = p.S;
     const int nq = (S + BM - 1) / BM;
 
-    const uint32_t sK = base + OFF_K, sV = base + OFF_V, sQ = base + OFF_Q, sDO = base + OFF_DO;
+    const uint32_t sK = base + OFF_K, sV = base + OFF_V;
+    auto sQ = [&](int s) { return base + OFF_STAGE + s * STAGE_BYTES; };
+    auto sDO = [&](int s) { return base + OFF_STAGE + s * STAGE_BYTES + TILE_BYTES; };
     const uint32_t bar0 = base + OFF_BAR;
     auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
@@ -114,7 +119,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         mbar_init(bar(KV_FULL), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(QDO_FULL + s), 1);
-            mbar_init(bar(QDO_EMPTY + s), 1);
+            mbar_init(bar(QDO_EMPTY + s), 2);    // the MMAs' commit + the dQ reducer's read-out
         }
         mbar_init(bar(S_FULL), 1);
         mbar_init(bar(DP_FULL), 1);
@@ -125,6 +130,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         mbar_init(bar(DQ_DRAINED), BM);
         mbar_init(bar(FINAL), 1);
         mbar_init(bar(DRAIN), 1);
+        mbar_init(bar(STAGED), BM);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -159,10 +165,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (!ok) break;
                 const uint32_t fb = bar(QDO_FULL + s);
                 mbar_arrive_expect_tx(fb, 2 * TILE_BYTES);
-                tma_load_4d_hint(sQ + s * TILE_BYTES, &tmq, fb, 0, h, i * BM, b, keep);
-                tma_load_4d_hint(sQ + s * TILE_BYTES + HALF_BYTES, &tmq, fb, 64, h, i * BM, b, keep);
-                tma_load_4d_hint(sDO + s * TILE_BYTES, &tmdo, fb, 0, h, i * BM, b, keep);
-                tma_load_4d_hint(sDO + s * TILE_BYTES + HALF_BYTES, &tmdo, fb, 64, h, i * BM, b, keep);
+                tma_load_4d_hint(sQ(s), &tmq, fb, 0, h, i * BM, b, keep);
+                tma_load_4d_hint(sQ(s) + HALF_BYTES, &tmq, fb, 64, h, i * BM, b, keep);
+                tma_load_4d_hint(sDO(s), &tmdo, fb, 0, h, i * BM, b, keep);
+                tma_load_4d_hint(sDO(s) + HALF_BYTES, &tmdo, fb, 64, h, i * BM, b, keep);
                 par[s] = use;
             }
             if (!ok) {
@@ -184,7 +190,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (ok && i > 0) ok = wait_thread(bar(DQ_DRAINED), (i - 1) & 1, wc);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t q_s = sQ + s * TILE_BYTES, do_s = sDO + s * TILE_BYTES;
+                const uint32_t q_s = sQ(s), do_s = sDO(s);
                 mma_kmajor(tmem + T_S, sK, q_s, id_kk, false);        // S^T = K Q^T
                 mma_commit(bar(S_FULL));
                 mma_kmajor(tmem + T_DP, sV, do_s, id_kk, false);      // dP^T = V dO^T
@@ -205,6 +211,20 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             if (ok) mma_commit(bar(FINAL));
             mma_commit(bar(DRAIN));
             drain_wait(bar(DRAIN), 0, p.wait_budget_ns);
+        }
+    } else if (warp == 6) {
+        // ------------------ dQ reducer: TMA reduce-add of each dQ tile ------------
+        if (lane == 0) {
+            bool ok = true;
+            for (int i = 0; i < nq && ok; ++i) {
+                ok = wait_thread(bar(STAGED), i & 1, wc);
+                if (!ok) break;
+                tma_reduce_add_4d(&tmdq, base + OFF_STAGE + (i & 1) * STAGE_BYTES, 0, h, i * BM, b);
+                bulk_commit_group();
+                bulk_wait_read_all();                         // the stage may be refilled now
+                mbar_arrive(bar(QDO_EMPTY + (i & 1)));
+            }
+            bulk_wait_all();
         }
     } else {
         // -------------------- gradients warpgroup (thread = key row / d) -----------
@@ -256,7 +276,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             ok = wait_warp(bar(DP_FULL), i & 1, wc) && wait_warp(bar(DV_DONE), i & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            uint8_t* ds_row = smem + OFF_DO + (i & 1) * TILE_BYTES + j * 128;   // row j of both halves
+            uint8_t* ds_row = smem + OFF_STAGE + (i & 1) * STAGE_BYTES + TILE_BYTES + j * 128;   // row j
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t dp[32];
@@ -288,23 +308,22 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             ok = wait_warp(bar(DQ_FULL), i & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            // dQ^T: TMEM lane = d (this thread's j), column = query within the tile
-            float* dq_col = p.dq_acc + h * HD + j;
+            // dQ^T: TMEM lane = d (this thread's j), column = query within the tile.  Copy it
+            // into the stage as fp32 [query][d] (the Q and dS^T it held are consumed), free the
+            // TMEM columns, and let the reducer warp add the tile into the accumulator by TMA.
+            float* stage = reinterpret_cast<float*>(smem + OFF_STAGE + (i & 1) * STAGE_BYTES);
 #pragma unroll 1
             for (int q = 0; q < 4; ++q) {
                 uint32_t v[32];
                 tmem_ld32(tS + q * 32, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int query = i * BM + q * 32 + e;
-                    if (query < S)
-                        atomicAdd(dq_col + (static_cast<size_t>(b) * S + query) * (static_cast<size_t>(p.H) * HD),
-                                  __uint_as_float(v[e]));
-                }
+                for (int e = 0; e < 32; ++e) stage[(q * 32 + e) * HD + j] = __uint_as_float(v[e]);
             }
             tc_fence_before();
             mbar_arrive(bar(DQ_DRAINED));
+            fence_async_smem();
+            mbar_arrive(bar(STAGED));
         }
         if (ok) ok = wait_warp(bar(FINAL), 0, wc);
         if (ok) {
@@ -407,7 +426,8 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ a
 }  // namespace bwd
 
 int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-               const BwdParams& p, const void* o, const void* dout, void* dq, cudaStream_t stream) {
+               const CUtensorMap& tdq, const BwdParams& p, const void* o, const void* dout, void* dq,
+               cudaStream_t stream) {
     const long long rows = static_cast<long long>(p.B) * p.S * p.H;
     int sms = 148;
     int dev = 0;
@@ -419,7 +439,7 @@ int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
     if (cudaGetLastError() != cudaSuccess) return -1;
     if (configure_smem(reinterpret_cast<const void*>(bwd::bwd_main_kernel), bwd::SMEM_BYTES) != 0) return -1;
     const dim3 grid((p.S + bwd::BM - 1) / bwd::BM, p.H, p.B);
-    bwd::bwd_main_kernel<<<grid, bwd::NTHREADS, bwd::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    bwd::bwd_main_kernel<<<grid, bwd::NTHREADS, bwd::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
     if (cudaGetLastError() != cudaSuccess) return -1;
     bwd::bwd_dq_kernel<<<ew_blocks, 256, 0, stream>>>(p.dq_acc, static_cast<__nv_bfloat16*>(dq), rows * 16,
                                                       p.scale);

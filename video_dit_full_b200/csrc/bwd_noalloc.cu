@@ -12,7 +12,7 @@
 
 #include <mutex>
 
-#include "../../include/wan_attn.h"
+#include "wan_attn.h"
 
 namespace {
 

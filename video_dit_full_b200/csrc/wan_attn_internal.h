@@ -60,7 +60,8 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
                cudaStream_t stream);
 
 int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-               const BwdParams& p, const void* o, const void* dout, void* dq, cudaStream_t stream);
+               const CUtensorMap& tdq, const BwdParams& p, const void* o, const void* dout, void* dq,
+               cudaStream_t stream);
 
 int launch_q8(const Q8QuantParams& qp, const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv8,
               const Q8AttnParams& p, cudaStream_t stream);
