@@ -8,7 +8,8 @@
 //
 // Three kernels:
 //   bwd_prep    D_i = sum_d dO_id O_id (fp32) and zeroing of the fp32 dQ accumulator.
-//   bwd_main    one CTA per 128-key tile of one (batch, head); K_j, V_j stay in
+//   bwd_main    one CTA per 128-key tile of one (batch, head), eight gradient warps (two
+//               threads per key row); K_j, V_j stay in
 //               shared memory while the CTA walks every 128-row Q tile i:
 //                 S^T = K Q_i^T, dP^T = V dO_i^T            (tcgen05, TMEM)
 //                 P^T = exp2(S^T c - lse_i log2 e)          (softmax warpgroup)
@@ -38,16 +39,20 @@ constexpr int OFF_V = OFF_K + TILE_BYTES;
 // after the dK and dQ MMAs the whole stage holds the fp32 dQ^T tile [query][d] for the TMA reduce.
 constexpr int OFF_STAGE = OFF_V + TILE_BYTES;
 constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-constexpr int OFF_VEC = OFF_STAGE + 2 * STAGE_BYTES;   // per warp: 128 fp32 lse*log2(e), 128 fp32 D_i
-constexpr int VEC_BYTES = 2 * BM * 4;
-constexpr int OFF_BAR = OFF_VEC + 4 * VEC_BYTES;
+constexpr int OFF_VEC = OFF_STAGE + 2 * STAGE_BYTES;   // per warp: 64 fp32 lse*log2(e), 64 fp32 D_i
+constexpr int VEC_BYTES = 2 * 64 * 4;
+constexpr int OFF_BAR = OFF_VEC + 8 * VEC_BYTES;
 enum Bar { KV_FULL = 0, QDO_FULL = 1, QDO_EMPTY = 3, S_FULL = 5, DP_FULL = 6, P_READY = 7, DV_DONE = 8,
            DS_READY = 9, DQ_FULL = 10, DQ_DRAINED = 11, FINAL = 12, DRAIN = 13, STAGED = 14, NBARS = 15 };
 constexpr int OFF_TMEM_SLOT = OFF_BAR + NBARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
 constexpr int SMEM_USED = OFF_ABORT + 8;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
-constexpr int NTHREADS = 224;            // warps 0-3 gradients, 4 TMA, 5 MMA, 6 dQ reducer
+// warps 0-7 gradients (two threads per key row: warps 0-3 take queries 0-63 of a tile,
+// warps 4-7 queries 64-127), 8 TMA, 9 MMA, 10 dQ reducer
+constexpr int NTHREADS = 352;
+constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_RED = 10;
+constexpr int G_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;      // S^T | dP^T | dV | dK
 constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -68,12 +73,14 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_smem, uin
 }
 
 // A in TMEM (bf16, 128 x 128), B MN-major in shared memory: K = the 128 rows of the B tile.
+// A's columns for K = 0-63 start at a_tmem, those for K = 64-127 at a_tmem + 64 (each half of
+// the row is written by its own thread into the TMEM columns it has just read).
 __device__ __forceinline__ void mma_ts_bmn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, uint32_t idesc,
                                            bool accumulate) {
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-        mma_f16_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc,
-                   (accumulate || kk > 0) ? 1u : 0u);
+        mma_f16_ts(d_tmem, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8, sdesc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024),
+                   idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // A and B both MN-major in shared memory, K = the 128 rows of both tiles.
@@ -123,18 +130,18 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         }
         mbar_init(bar(S_FULL), 1);
         mbar_init(bar(DP_FULL), 1);
-        mbar_init(bar(P_READY), BM);
+        mbar_init(bar(P_READY), G_THREADS);
         mbar_init(bar(DV_DONE), 1);
-        mbar_init(bar(DS_READY), BM);
+        mbar_init(bar(DS_READY), G_THREADS);
         mbar_init(bar(DQ_FULL), 1);
-        mbar_init(bar(DQ_DRAINED), BM);
+        mbar_init(bar(DQ_DRAINED), G_THREADS);
         mbar_init(bar(FINAL), 1);
         mbar_init(bar(DRAIN), 1);
-        mbar_init(bar(STAGED), BM);
+        mbar_init(bar(STAGED), G_THREADS);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == WARP_MMA) {
         tmem_alloc(base + OFF_TMEM_SLOT, TMEM_COLS);
         tmem_relinquish();
     }
@@ -143,7 +150,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
 
-    if (warp == 4) {
+    if (warp == WARP_TMA) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
             tma_prefetch_desc(&tmq);
@@ -177,7 +184,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     if (par[s] >= 0) drain_wait(bar(QDO_FULL + s), par[s], p.wait_budget_ns);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == WARP_MMA) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
             const uint32_t id_kk = make_idesc(1, 1, 1, 0, 0, BM, BM);   // both K-major
@@ -212,7 +219,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             mma_commit(bar(DRAIN));
             drain_wait(bar(DRAIN), 0, p.wait_budget_ns);
         }
-    } else if (warp == 6) {
+    } else if (warp == WARP_RED) {
         // ------------------ dQ reducer: TMA reduce-add of each dQ tile ------------
         if (lane == 0) {
             bool ok = true;
@@ -227,24 +234,29 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             bulk_wait_all();
         }
     } else {
-        // -------------------- gradients warpgroup (thread = key row / d) -----------
-        const int j = threadIdx.x;                         // 0..127
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t tS = tmem + T_S + lane_off, tDP = tmem + T_DP + lane_off;
+        // -------- gradient warps: two threads per key row (or per d for dQ^T) -------
+        // Thread (j, hq): key row / TMEM lane j = 32*(warp%4) + lane; query half hq = warp/4
+        // covers queries 64hq..64hq+63 of each Q tile.  It writes P^T and dS^T (bf16) into the
+        // first 32 of the 64 TMEM columns it has just read, so the halves never race.
+        const int hq = warp >> 2;
+        const int cb = hq * 64;                            // first query column of this half
+        const int j = (warp & 3) * 32 + lane;              // 0..127
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + T_S + lane_off + cb, tDP = tmem + T_DP + lane_off + cb;
         const int key = kv0 + j;
         const bool key_ok = key < S;
         const float c = p.scale_log2;
         const size_t bh = static_cast<size_t>(b) * p.H + h;
-        // each warp keeps its own copy of the Q tile's lse / D (no cross-warp barrier needed)
+        // each warp keeps its own copy of its 64 queries' lse / D (no cross-warp barrier needed)
         float* s_lse = reinterpret_cast<float*>(smem + OFF_VEC + warp * VEC_BYTES);
-        float* s_del = s_lse + BM;
+        float* s_del = s_lse + 64;
         bool ok = true;
         for (int i = 0; i < nq && ok; ++i) {
             __syncwarp();                                    // previous tile's values no longer read
 #pragma unroll
-            for (int e = 0; e < BM / 32; ++e) {
+            for (int e = 0; e < 2; ++e) {
                 const int col = e * 32 + lane;
-                const int qi = i * BM + col;
+                const int qi = i * BM + cb + col;
                 s_lse[col] = qi < S ? p.lse[bh * S + qi] * LOG2E : INFINITY;
                 s_del[col] = qi < S ? p.delta[bh * S + qi] : 0.f;
             }
@@ -253,21 +265,20 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             ok = wait_warp(bar(S_FULL), i & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            float pr[128];
+            float pr[64];
             {
                 uint32_t* sr = reinterpret_cast<uint32_t*>(pr);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q * 32]));
+                tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                 tmem_wait_ld();
             }
 #pragma unroll
-            for (int e = 0; e < 128; ++e) pr[e] = key_ok ? ex2_approx(fmaf(pr[e], c, -s_lse[e])) : 0.f;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            for (int e = 0; e < 64; ++e) pr[e] = key_ok ? ex2_approx(fmaf(pr[e], c, -s_lse[e])) : 0.f;
+            {
                 uint32_t pk[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[half * 64 + 2 * e], pr[half * 64 + 2 * e + 1]);
-                tmem_st32(tS + half * 32, pk);
+                for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+                tmem_st32(tS, pk);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -276,9 +287,10 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             ok = wait_warp(bar(DP_FULL), i & 1, wc) && wait_warp(bar(DV_DONE), i & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            uint8_t* ds_row = smem + OFF_STAGE + (i & 1) * STAGE_BYTES + TILE_BYTES + j * 128;   // row j
+            // dS^T row j, queries cb..cb+63 -> the 128-byte swizzled row j of half hq (in dO's buffer)
+            uint8_t* half_row = smem + OFF_STAGE + (i & 1) * STAGE_BYTES + TILE_BYTES + hq * HALF_BYTES + j * 128;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 uint32_t dp[32];
                 tmem_ld32(tDP + q * 32, dp);
                 tmem_wait_ld();
@@ -291,11 +303,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     pk[e] = pack_bf16x2(d0, d1);
                 }
                 tmem_st16(tDP + q * 16, pk);
-                // dS^T row j, queries 32q..32q+31 -> 128-byte swizzled row of half q/2
-                uint8_t* half_row = ds_row + (q >> 1) * HALF_BYTES;
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) {
-                    const int chunk = ((q & 1) * 4 + ch) ^ (j & 7);
+                    const int chunk = (q * 4 + ch) ^ (j & 7);
                     *reinterpret_cast<uint4*>(half_row + chunk * 16) =
                         make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
                 }
@@ -308,17 +318,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             ok = wait_warp(bar(DQ_FULL), i & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            // dQ^T: TMEM lane = d (this thread's j), column = query within the tile.  Copy it
-            // into the stage as fp32 [query][d] (the Q and dS^T it held are consumed), free the
-            // TMEM columns, and let the reducer warp add the tile into the accumulator by TMA.
+            // dQ^T: TMEM lane = d (= j), column = query.  Copy queries cb..cb+63 into the stage as
+            // fp32 [query][d] (its Q and dS^T are consumed), free the TMEM columns, and let the
+            // reducer warp add the tile into the accumulator by TMA.
             float* stage = reinterpret_cast<float*>(smem + OFF_STAGE + (i & 1) * STAGE_BYTES);
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 uint32_t v[32];
                 tmem_ld32(tS + q * 32, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) stage[(q * 32 + e) * HD + j] = __uint_as_float(v[e]);
+                for (int e = 0; e < 32; ++e) stage[(cb + q * 32 + e) * HD + j] = __uint_as_float(v[e]);
             }
             tc_fence_before();
             mbar_arrive(bar(DQ_DRAINED));
@@ -328,14 +338,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         if (ok) ok = wait_warp(bar(FINAL), 0, wc);
         if (ok) {
             tc_fence_after();
-            const size_t row = ((static_cast<size_t>(b) * S + key) * p.H + h) * HD;
+            const size_t row = ((static_cast<size_t>(b) * S + key) * p.H + h) * HD + cb;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
-                const uint32_t src = tmem + (which ? T_DK : T_DV) + lane_off;
+                const uint32_t src = tmem + (which ? T_DK : T_DV) + lane_off + cb;
                 const float mul = which ? p.scale : 1.f;
                 __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(which ? p.dk : p.dv) + row;
 #pragma unroll 1
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
                     uint32_t v[32];
                     tmem_ld32(src + q * 32, v);
                     tmem_wait_ld();
@@ -357,7 +367,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == WARP_MMA) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 // D_i = sum_d dO_id * O_id (fp32) for every (b, s, h) row, and dQ accumulator := 0.
