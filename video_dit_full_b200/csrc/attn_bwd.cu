@@ -43,7 +43,8 @@ constexpr int OFF_VEC = OFF_STAGE + 2 * STAGE_BYTES;   // per warp: 64 fp32 lse*
 constexpr int VEC_BYTES = 2 * 64 * 4;
 constexpr int OFF_BAR = OFF_VEC + 8 * VEC_BYTES;
 enum Bar { KV_FULL = 0, QDO_FULL = 1, QDO_EMPTY = 3, S_FULL = 5, DP_FULL = 6, P_READY = 7, DV_DONE = 8,
-           DS_READY = 9, DQ_FULL = 10, DQ_DRAINED = 11, FINAL = 12, DRAIN = 13, STAGED = 14, NBARS = 15 };
+           DS_READY = 9, DQ_FULL = 10, DQ_DRAINED = 11, FINAL = 12, DRAIN = 13, STAGED = 14, DS_SMEM = 15,
+           NBARS = 16 };
 constexpr int OFF_TMEM_SLOT = OFF_BAR + NBARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
 constexpr int SMEM_USED = OFF_ABORT + 8;
@@ -132,7 +133,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         mbar_init(bar(DP_FULL), 1);
         mbar_init(bar(P_READY), G_THREADS);
         mbar_init(bar(DV_DONE), 1);
-        mbar_init(bar(DS_READY), G_THREADS);
+        mbar_init(bar(DS_READY), G_THREADS);     // dS^T in TMEM (dK may start)
+        mbar_init(bar(DS_SMEM), G_THREADS);      // dS^T in shared memory (dQ may start)
         mbar_init(bar(DQ_FULL), 1);
         mbar_init(bar(DQ_DRAINED), G_THREADS);
         mbar_init(bar(FINAL), 1);
@@ -211,6 +213,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (!ok) break;
                 tc_fence_after();
                 mma_ts_bmn(tmem + T_DK, tmem + T_DP, q_s, id_tb, i > 0);   // dK += dS^T Q
+                ok = wait_thread(bar(DS_SMEM), i & 1, wc);
+                if (!ok) break;
                 mma_ss_mn(tmem + T_S, sK, do_s, id_mm);                    // dQ^T = K^T dS^T (dS^T in dO's buffer)
                 mma_commit(bar(DQ_FULL));
                 mma_commit(bar(QDO_EMPTY + s));
@@ -284,36 +288,37 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             tc_fence_before();
             mbar_arrive(bar(P_READY));
 
-            ok = wait_warp(bar(DP_FULL), i & 1, wc) && wait_warp(bar(DV_DONE), i & 1, wc);
+            ok = wait_warp(bar(DP_FULL), i & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            // dS^T row j, queries cb..cb+63 -> the 128-byte swizzled row j of half hq (in dO's buffer)
-            uint8_t* half_row = smem + OFF_STAGE + (i & 1) * STAGE_BYTES + TILE_BYTES + hq * HALF_BYTES + j * 128;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                uint32_t dp[32];
-                tmem_ld32(tDP + q * 32, dp);
+            uint32_t dsp[32];                                // this half-row's dS^T, bf16 pairs
+            {
+                uint32_t dp[64];
+                tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+                tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
                 tmem_wait_ld();
-                uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int c0 = q * 32 + 2 * e;
-                    const float d0 = pr[c0] * (__uint_as_float(dp[2 * e]) - s_del[c0]);
-                    const float d1 = pr[c0 + 1] * (__uint_as_float(dp[2 * e + 1]) - s_del[c0 + 1]);
-                    pk[e] = pack_bf16x2(d0, d1);
-                }
-                tmem_st16(tDP + q * 16, pk);
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const int chunk = (q * 4 + ch) ^ (j & 7);
-                    *reinterpret_cast<uint4*>(half_row + chunk * 16) =
-                        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+                for (int e = 0; e < 32; ++e) {
+                    const float d0 = pr[2 * e] * (__uint_as_float(dp[2 * e]) - s_del[2 * e]);
+                    const float d1 = pr[2 * e + 1] * (__uint_as_float(dp[2 * e + 1]) - s_del[2 * e + 1]);
+                    dsp[e] = pack_bf16x2(d0, d1);
                 }
             }
+            tmem_st32(tDP, dsp);
             tmem_wait_st();
-            fence_async_smem();
             tc_fence_before();
             mbar_arrive(bar(DS_READY));
+            // dS^T row j, queries cb..cb+63 -> the 128-byte swizzled row j of half hq, in dO's
+            // buffer: only once dV (the last reader of dO) is done
+            ok = wait_warp(bar(DV_DONE), i & 1, wc);
+            if (!ok) break;
+            uint8_t* half_row = smem + OFF_STAGE + (i & 1) * STAGE_BYTES + TILE_BYTES + hq * HALF_BYTES + j * 128;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(half_row + ((ch ^ (j & 7)) * 16)) =
+                    make_uint4(dsp[4 * ch], dsp[4 * ch + 1], dsp[4 * ch + 2], dsp[4 * ch + 3]);
+            fence_async_smem();
+            mbar_arrive(bar(DS_SMEM));
 
             ok = wait_warp(bar(DQ_FULL), i & 1, wc);
             if (!ok) break;
