@@ -57,6 +57,10 @@ constexpr int G_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;      // S^T | dP^T | dV | dK
 constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
 constexpr float LOG2E = 1.4426950408889634f;
+#ifndef WAN_BWD_POLY_PAIRS
+#define WAN_BWD_POLY_PAIRS 2          // of every 8 pairs of exponentials in P, this many use exp2_poly3
+#endif
+constexpr int BWD_POLY_PAIRS = WAN_BWD_POLY_PAIRS;
 
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -277,7 +281,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 tmem_wait_ld();
             }
 #pragma unroll
-            for (int e = 0; e < 64; ++e) pr[e] = key_ok ? ex2_approx(fmaf(pr[e], c, -s_lse[e])) : 0.f;
+            for (int e = 0; e < 64; ++e) {
+                // a share of the exponentials runs on the FMA pipe (the MUFU bounds this phase)
+                const float x = fmaf(pr[e], c, -s_lse[e]);
+                const float pe = ((e >> 1) & 7) < BWD_POLY_PAIRS ? exp2_poly3(x) : ex2_approx(x);
+                pr[e] = key_ok ? pe : 0.f;
+            }
             {
                 uint32_t pk[32];
 #pragma unroll
