@@ -12,8 +12,9 @@
 //                 codes (IEEE division, round to nearest even), written
 //                 head-major [B, H, S, 128] into the workspace.
 //   q8_attn       one CTA per 128-row Q tile of one (b, h), 128-key K/V tiles:
-//                 warp 8 TMA, warp 9 tcgen05 issuer, warps 0-3 softmax (one row
-//                 per thread), warps 4-7 fp32 accumulation of O (one row per thread).
+//                 warp 16 TMA, warp 17 tcgen05 issuer, warps 0-7 softmax (two threads
+//                 per row, one 64-key block each, partial maxima swapped through
+//                 shared memory), warps 8-15 fp32 accumulation of O (two per row).
 //                   S = Q8 K8^T          kind::i8, int32 in TMEM (two buffers)
 //                   s = S sQ sK / sqrt(D) * log2(e) per 64-key column block
 //                   P8 = e4m3(2^(s - m + log2 448)) -> TMEM (over S)
@@ -125,14 +126,24 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + T8;
 constexpr int OFF_V = OFF_K + STAGES * T8;
 constexpr int OFF_ALPHA = OFF_V + STAGES * T8;        // 4 x 128 fp32 rescale factors
-constexpr int OFF_STAT = OFF_ALPHA + 4 * BM * 4;      // final m, l per row
-constexpr int OFF_BAR = OFF_STAT + 2 * BM * 4;
+constexpr int OFF_STAT = OFF_ALPHA + 4 * BM * 4;      // final m per row, l per (half, row)
+constexpr int OFF_XMAX = OFF_STAT + 3 * BM * 4;       // [parity][half][row] partial row maxima
+constexpr int OFF_BAR = OFF_XMAX + 2 * 2 * BM * 4;
 enum Bar { Q_FULL = 0, K_FULL = 1, K_EMPTY = 4, V_FULL = 7, V_EMPTY = 10, S_FULL = 13, P_READY = 15,
-           ALPHA_READY = 17, OB_FULL = 21, OB_FREE = 22, STATS = 23, DRAIN = 24, NBARS = 25 };
+           ALPHA_READY = 17, OB_FULL = 21, OB_FREE = 22, STATS = 23, DRAIN = 24, XCHG = 25, NBARS = 27 };
 constexpr int OFF_TMEM_SLOT = OFF_BAR + NBARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
 constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
-constexpr int NTHREADS = 320;
+// warps 0-7 softmax (two threads per row: warps 0-3 keys 0-63 of a tile = one quantisation
+// block, warps 4-7 keys 64-127), warps 8-15 fp32 accumulation of O (two threads per row:
+// d 0-63 / 64-127), 16 TMA, 17 MMA
+constexpr int NTHREADS = 576;
+constexpr int WARP_TMA = 16, WARP_MMA = 17;
+constexpr int HALF_THREADS = 256;
+#ifndef WAN_Q8_POLY_PAIRS
+#define WAN_Q8_POLY_PAIRS 0            // of every 8 pairs of exponentials, this many use exp2_poly3
+#endif
+constexpr int Q8_POLY_PAIRS = WAN_Q8_POLY_PAIRS;
 constexpr uint32_t TMEM_COLS = 512;         // S0 | S1 (int32, P8 over the first 32 columns) | Ob_a | Ob_b
 constexpr uint32_t T_OBA = 256, T_OBB = 384;
 constexpr float LOG2_448 = 8.807354922057604f;
@@ -152,14 +163,15 @@ __device__ __forceinline__ void issue_qk8(uint32_t d_tmem, uint32_t q_smem, uint
                   idesc, kk > 0 ? 1u : 0u);
 }
 
-// Ob_a, Ob_b = P8 V8 for keys 0-63 and 64-127 of the tile; P8 in TMEM (4 per column),
+// Ob_a, Ob_b = P8 V8 for keys 0-63 and 64-127 of the tile; P8 in TMEM (4 per column; keys
+// 0-63 at columns 0-15, keys 64-127 at columns 64-79, each written by the thread that read them),
 // V8 [key][d] MN-major (one 128-byte swizzle atom spans all 128 d), 32 keys per MMA.
 __device__ __forceinline__ void issue_pv8(uint32_t tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc) {
 #pragma unroll
     for (int a = 0; a < 2; ++a) {
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
-            mma_f8_ts(tmem + (a ? T_OBB : T_OBA), p_tmem + a * 16 + kk * 8,
+            mma_f8_ts(tmem + (a ? T_OBB : T_OBA), p_tmem + a * 64 + kk * 8,
                       sdesc_sw128(v_smem + a * 8192 + kk * 4096, 16, 1024), idesc, kk > 0 ? 1u : 0u);
     }
 }
@@ -183,7 +195,7 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sV = base + OFF_V;
     float* alpha_buf = reinterpret_cast<float*>(smem + OFF_ALPHA);
     float* stat_m = reinterpret_cast<float*>(smem + OFF_STAT);
-    float* stat_l = stat_m + BM;
+    float* stat_l = stat_m + BM;                           // [half][row]
     const uint32_t bar0 = base + OFF_BAR;
     auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
@@ -199,17 +211,18 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(S_FULL + s), 1);
-            mbar_init(bar(P_READY + s), BM);
+            mbar_init(bar(P_READY + s), HALF_THREADS);
+            mbar_init(bar(XCHG + s), HALF_THREADS);
         }
-        for (int s = 0; s < 4; ++s) mbar_init(bar(ALPHA_READY + s), BM);
+        for (int s = 0; s < 4; ++s) mbar_init(bar(ALPHA_READY + s), HALF_THREADS);
         mbar_init(bar(OB_FULL), 1);
-        mbar_init(bar(OB_FREE), BM);
-        mbar_init(bar(STATS), BM);
+        mbar_init(bar(OB_FREE), HALF_THREADS);
+        mbar_init(bar(STATS), HALF_THREADS);
         mbar_init(bar(DRAIN), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 9) {
+    if (warp == WARP_MMA) {
         tmem_alloc(base + OFF_TMEM_SLOT, TMEM_COLS);
         tmem_relinquish();
     }
@@ -218,7 +231,7 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
 
-    if (warp == 8) {
+    if (warp == WARP_TMA) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
             tma_prefetch_desc(&tmq);
@@ -251,7 +264,7 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 }
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == WARP_MMA) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
             const uint32_t idesc_qk = make_idesc(2, 1, 1, 0, 0, BM, BN);   // s32 <- s8 x s8
@@ -289,78 +302,98 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             mma_commit(bar(DRAIN));
             drain_wait(bar(DRAIN), 0, p.wait_budget_ns);
         }
-    } else if (warp < 4) {
-        // ------------------------------ softmax (row r) ---------------------------
-        const int r = threadIdx.x;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    } else if (warp < 8) {
+        // ------------------- softmax (row r, key half hc = one 64-key block) -------
+        const int hc = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const int row = q0 + r;
         const float* sk = p.sk + static_cast<size_t>(bh) * p.nblk;
         const float sq_row = p.sq[static_cast<size_t>(bh) * p.nblk + min(row, S - 1) / BLK];
+        float* xmax = reinterpret_cast<float*>(smem + OFF_XMAX);
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nkv && ok; ++j) {
             const int sb = j & 1;
+            const int kb = 2 * j + hc;                      // this thread's quantisation block
             ok = wait_warp(bar(S_FULL + sb), (j >> 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            uint32_t sr[128];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                tmem_ld32(tmem + sb * BN + lane_off + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q * 32]));
+            const uint32_t tS = tmem + sb * BN + lane_off + hc * 64;
+            uint32_t sr[64];
+            tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
             tmem_wait_ld();
-            const int kb = 2 * j;
-            const float ca = sq_row * sk[kb] * p.scale_log2;
-            const float cb = kb + 1 < p.nblk ? sq_row * sk[kb + 1] * p.scale_log2 : 0.f;
+            const float cs = kb < p.nblk ? sq_row * sk[kb] * p.scale_log2 : 0.f;
             float* s = reinterpret_cast<float*>(sr);
             // int32 -> fp32 without the conversion unit: |S| <= 128*127*127 < 2^22, so
             // adding 1.5*2^23 as a float bit pattern and subtracting it back is exact.
 #pragma unroll
-            for (int c = 0; c < 128; ++c)
-                s[c] = (__int_as_float(static_cast<int>(sr[c]) + 0x4B400000) - 12582912.f) * (c < 64 ? ca : cb);
-            const int valid = S - j * BN;
-            if (valid < BN) {
+            for (int c = 0; c < 64; ++c)
+                s[c] = (__int_as_float(static_cast<int>(sr[c]) + 0x4B400000) - 12582912.f) * cs;
+            const int valid = S - j * BN - hc * 64;
+            if (valid < 64) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
+                for (int c = 0; c < 64; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            float m8[8];
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            for (int c = 0; c < 8; ++c) m8[c] = s[c];
+#pragma unroll
+            for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+#pragma unroll
+            for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                for (int c = 0; c < w; ++c) m8[c] = fmaxf(m8[c], m8[c + w]);
+            // swap partial maxima with the other half of the row
+            const int xb = (sb * 2) * BM;
+            xmax[xb + hc * BM + r] = m8[0];
+            mbar_arrive(bar(XCHG + sb));
+            ok = wait_warp(bar(XCHG + sb), (j >> 1) & 1, wc);
+            if (!ok) break;
+            const float mx = fmaxf(m8[0], xmax[xb + (hc ^ 1) * BM + r]);
             const float m_new = fmaxf(m, mx);
             const float alpha = ex2_approx(m - m_new);
             const float bias = m_new - LOG2_448;       // p * 448 = 2^(s - bias) <= 448
-            float sum = 0.f;
-            uint32_t pk[32];
+            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[16];
 #pragma unroll
-            for (int w = 0; w < 32; ++w) {
-                const float p0 = ex2_approx(s[4 * w] - bias), p1 = ex2_approx(s[4 * w + 1] - bias);
-                const float p2 = ex2_approx(s[4 * w + 2] - bias), p3 = ex2_approx(s[4 * w + 3] - bias);
-                sum += (p0 + p1) + (p2 + p3);
+            for (int w = 0; w < 16; ++w) {
+                const bool poly = ((2 * w) & 7) < 2 * Q8_POLY_PAIRS;
+                const float x0 = s[4 * w] - bias, x1 = s[4 * w + 1] - bias;
+                const float x2 = s[4 * w + 2] - bias, x3 = s[4 * w + 3] - bias;
+                const float p0 = poly ? exp2_poly3(x0) : ex2_approx(x0);
+                const float p1 = poly ? exp2_poly3(x1) : ex2_approx(x1);
+                const float p2 = poly ? exp2_poly3(x2) : ex2_approx(x2);
+                const float p3 = poly ? exp2_poly3(x3) : ex2_approx(x3);
+                sum4[w & 3] += (p0 + p1) + (p2 + p3);
                 pk[w] = pack_e4m3x2(p0, p1) | (pack_e4m3x2(p2, p3) << 16);
             }
-            tmem_st32(tmem + sb * BN + lane_off, pk);
-            l = l * alpha + sum;
+            tmem_st16(tS, pk);                                 // P8 over the columns this thread read
+            l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
             m = m_new;
-            alpha_buf[(j & 3) * BM + r] = alpha;
+            if (hc == 0) alpha_buf[(j & 3) * BM + r] = alpha;
             mbar_arrive(bar(ALPHA_READY + (j & 3)));
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(P_READY + sb));
         }
         if (ok) {
-            stat_m[r] = m;
-            stat_l[r] = l;
+            if (hc == 0) stat_m[r] = m;
+            stat_l[hc * BM + r] = l;
             mbar_arrive(bar(STATS));
         }
     } else {
-        // --------------------- fp32 accumulation of O (row r) -----------------------
-        const int r = threadIdx.x - 128;
+        // ------------- fp32 accumulation of O (row r, d half hd) -----------------
+        const int hd = (warp >> 2) & 1;
+        const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const int row = q0 + r;
         const float* sv = p.sv + static_cast<size_t>(bh) * p.nblk;
-        float o[128];
+        float o[64];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) o[c] = 0.f;
+        for (int c = 0; c < 64; ++c) o[c] = 0.f;
         bool ok = true;
         for (int j = 0; j < nkv && ok; ++j) {
             ok = wait_warp(bar(ALPHA_READY + (j & 3)), (j >> 2) & 1, wc);
@@ -373,10 +406,10 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             const float sva = sv[kb];
             const float svb = kb + 1 < p.nblk ? sv[kb + 1] : 0.f;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < 4; ++q) {
                 uint32_t a[16], bb[16];
-                tmem_ld16(tmem + T_OBA + lane_off + q * 16, a);
-                tmem_ld16(tmem + T_OBB + lane_off + q * 16, bb);
+                tmem_ld16(tmem + T_OBA + lane_off + hd * 64 + q * 16, a);
+                tmem_ld16(tmem + T_OBB + lane_off + hd * 64 + q * 16, bb);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
@@ -388,25 +421,26 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         }
         if (ok) ok = wait_warp(bar(STATS), 0, wc);
         if (ok && row < S) {
-            const float m = stat_m[r], l = stat_l[r];
+            const float m = stat_m[r], l = stat_l[r] + stat_l[BM + r];
             const float inv_l = 1.f / l;
             __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                  ((static_cast<size_t>(b) * S + row) * p.H + h) * HD;
+                                  ((static_cast<size_t>(b) * S + row) * p.H + h) * HD + hd * 64;
             uint4* d4 = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
+            for (int u = 0; u < 8; ++u)
                 d4[u] = make_uint4(pack_bf16x2(o[8 * u] * inv_l, o[8 * u + 1] * inv_l),
                                    pack_bf16x2(o[8 * u + 2] * inv_l, o[8 * u + 3] * inv_l),
                                    pack_bf16x2(o[8 * u + 4] * inv_l, o[8 * u + 5] * inv_l),
                                    pack_bf16x2(o[8 * u + 6] * inv_l, o[8 * u + 7] * inv_l));
-            p.lse[static_cast<size_t>(bh) * S + row] = (m + log2f(l) - LOG2_448) * 0.69314718055994531f;
+            if (hd == 0)
+                p.lse[static_cast<size_t>(bh) * S + row] = (m + log2f(l) - LOG2_448) * 0.69314718055994531f;
         }
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 9) tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == WARP_MMA) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 }  // namespace q8
