@@ -33,7 +33,7 @@ METRIC = "attention TFLOP/s (4*B*H*S^2*D fwd)"
 
 # DRAM bytes (read + write) of one launch of the dominant kernel from an ncu
 # capture (profiles/), per workload; None where the kernel changed since.
-TRAFFIC = {"wan14b_720p": 3.335e9}
+TRAFFIC = {"wan14b_720p": 3.335e9, "train_480p_fwd_bwd": 3.54e9, "q8_720p": 1.94e9}
 
 
 def load_peaks():
@@ -154,6 +154,21 @@ def run_reference(args, w):
     return 0
 
 
+def max_over_ranks(ms: float, dist=None, device=None) -> float:
+    """The largest of every rank's device-timed milliseconds (all ranks take part)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flop_per_rank_step: float, steps: int, slowest_ms: float) -> float:
+    """Whole-job throughput: every rank's FLOPs over the slowest rank's time (weak scaling)."""
+    return world * flop_per_rank_step * steps / (slowest_ms * 1e-3) / 1e12
+
+
 class Path:
     """The calls one bench step makes for a workload, with their buffers.
 
@@ -254,13 +269,6 @@ def run_ours(args, w):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(ms):
-        if dist is None:
-            return ms
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # ------------------------ device-resident timing ------------------------
     for _ in range(args.warmup):
         path.step()
@@ -280,10 +288,10 @@ def run_ours(args, w):
     clocks = sampler.stop()
     barrier()
     status = status or wa.sync_status()
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
     dom_ms = [a.elapsed_time(b) for a, b in ev]
     ms_per_step = total_ms / args.steps
-    value = world * path.flop * args.steps / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, path.flop, args.steps, total_ms)
 
     # ------------------- end to end through host buffers ---------------------
     e2e_steps = max(1, min(args.steps, 5))
@@ -296,8 +304,8 @@ def run_ours(args, w):
         path.e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * path.flop * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    e2e_value = whole_job_tflops(world, path.flop, e2e_steps, e2e_ms)
     status = status or wa.sync_status()
 
     if rank == 0:
