@@ -96,13 +96,6 @@ __device__ __forceinline__ void mma_ss_mn(uint32_t d_tmem, uint32_t a_smem, uint
                    sdesc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc, kk > 0 ? 1u : 0u);
 }
 
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > budget_ns) break;
-    }
-}
-
 __global__ void __launch_bounds__(NTHREADS, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
@@ -185,9 +178,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 par[s] = use;
             }
             if (!ok) {
-                drain_wait(bar(KV_FULL), 0, p.wait_budget_ns);
+                drain_wait(bar(KV_FULL), 0);
                 for (int s = 0; s < 2; ++s)
-                    if (par[s] >= 0) drain_wait(bar(QDO_FULL + s), par[s], p.wait_budget_ns);
+                    if (par[s] >= 0) drain_wait(bar(QDO_FULL + s), par[s]);
             }
         }
     } else if (warp == WARP_MMA) {
@@ -225,7 +218,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             }
             if (ok) mma_commit(bar(FINAL));
             mma_commit(bar(DRAIN));
-            drain_wait(bar(DRAIN), 0, p.wait_budget_ns);
+            drain_wait(bar(DRAIN), 0);
         }
     } else if (warp == WARP_RED) {
         // ------------------ dQ reducer: TMA reduce-add of each dQ tile ------------

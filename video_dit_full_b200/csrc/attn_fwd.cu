@@ -68,14 +68,6 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
     }
 }
 
-// A wait used only while draining after an abort: ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > budget_ns) break;
-    }
-}
-
 __global__ void __launch_bounds__(NTHREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
@@ -153,10 +145,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             }
             if (!ok) {
                 // let the copies already issued land before the CTA's shared memory goes away
-                for (int t = 0; t < nq; ++t) drain_wait(bar(Q_FULL + t), 0, p.wait_budget_ns);
+                for (int t = 0; t < nq; ++t) drain_wait(bar(Q_FULL + t), 0);
                 for (int s = 0; s < 2; ++s) {
-                    if (kpar[s] >= 0) drain_wait(bar(K_FULL + s), kpar[s], p.wait_budget_ns);
-                    if (vpar[s] >= 0) drain_wait(bar(V_FULL + s), vpar[s], p.wait_budget_ns);
+                    if (kpar[s] >= 0) drain_wait(bar(K_FULL + s), kpar[s]);
+                    if (vpar[s] >= 0) drain_wait(bar(V_FULL + s), vpar[s]);
                 }
             }
         }
@@ -202,7 +194,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             }
             // every MMA issued so far completes before TMEM is released
             mma_commit(bar(DRAIN));
-            drain_wait(bar(DRAIN), 0, p.wait_budget_ns);
+            drain_wait(bar(DRAIN), 0);
         }
     } else {
         // ------------------------- softmax / correction / epilogue ----------------

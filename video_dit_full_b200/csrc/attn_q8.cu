@@ -148,13 +148,6 @@ constexpr uint32_t TMEM_COLS = 512;         // S0 | S1 (int32, P8 over the first
 constexpr uint32_t T_OBA = 256, T_OBB = 384;
 constexpr float LOG2_448 = 8.807354922057604f;
 
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > budget_ns) break;
-    }
-}
-
 // S (int32) = Q8 K8^T: both [128 rows][128 bytes] K-major with the 128-byte swizzle, K = 32 per MMA.
 __device__ __forceinline__ void issue_qk8(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem, uint32_t idesc) {
 #pragma unroll
@@ -257,10 +250,10 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 vpar[s] = use;
             }
             if (!ok) {
-                drain_wait(bar(Q_FULL), 0, p.wait_budget_ns);
+                drain_wait(bar(Q_FULL), 0);
                 for (int s = 0; s < STAGES; ++s) {
-                    if (kpar[s] >= 0) drain_wait(bar(K_FULL + s), kpar[s], p.wait_budget_ns);
-                    if (vpar[s] >= 0) drain_wait(bar(V_FULL + s), vpar[s], p.wait_budget_ns);
+                    if (kpar[s] >= 0) drain_wait(bar(K_FULL + s), kpar[s]);
+                    if (vpar[s] >= 0) drain_wait(bar(V_FULL + s), vpar[s]);
                 }
             }
         }
@@ -300,7 +293,7 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 }
             }
             mma_commit(bar(DRAIN));
-            drain_wait(bar(DRAIN), 0, p.wait_budget_ns);
+            drain_wait(bar(DRAIN), 0);
         }
     } else if (warp < 8) {
         // ------------------- softmax (row r, key half hc = one 64-key block) -------

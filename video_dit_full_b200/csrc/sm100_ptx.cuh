@@ -79,6 +79,19 @@ __device__ __forceinline__ bool wait_expired(const WaitCtl& w, uint64_t t0) {
     return false;
 }
 
+// Used only after an abort, to let the copies and MMAs a thread already issued
+// land before the CTA's shared and tensor memory go away.  It ignores the abort
+// flag and uses its own budget (those operations finish in microseconds; the
+// budget only bounds a GPU that has stopped making progress), so a tiny
+// user-set wait budget cannot cut it short.
+constexpr uint64_t kDrainBudgetNs = 50000000ull;   // 50 ms
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kDrainBudgetNs) break;
+    }
+}
+
 // One thread waits for the phase of `bar` with the given parity.  false = gave up.
 __device__ __forceinline__ bool wait_thread(uint32_t bar, uint32_t parity, const WaitCtl& w) {
     if (mbar_try_wait(bar, parity)) return true;
