@@ -108,13 +108,17 @@ WAN_ATTN_API size_t wan_attn_fwd_q8_workspace_size(int B, int S, int H, int D);
  * summary, section "干预与形式化": mixed int8/FP8 with FP32 accumulation
  * across blocks; kwkr.cn Wan explainer, section 4.2).  Read as:
  *   - per (b, h, 64-token block): sQ = absmax(Q)/127, sK = absmax(K)/127,
- *     sV = absmax(V)/448 (fp32; 1 for an all-zero block); codes
+ *     sV = the smallest power of two >= absmax(V)/448, at least 2^-126
+ *     (fp32; every scale is 1 for an all-zero block); codes
  *     Q8 = clamp(rint(q / sQ), -127, 127), K8 likewise, V8 = e4m3(v / sV),
  *     each division IEEE fp32, rounding to nearest even, e4m3 saturating;
  *   - scores S = (Q8 . K8) sQ sK / sqrt(D) from int32 tensor-core sums;
- *   - P8 = e4m3(448 * exp(S - running max)); each 64-key block's P8 V8
- *     product is taken out of the tensor core in fp32 and added to O with
- *     that block's sV; the row sum uses the unquantised exponentials.
+ *   - P8 = e4m3(224 * exp(S - m) * sV_block / sV_max), where m is the running
+ *     row max (moved only when it rises by more than a factor 2) and sV_max
+ *     the head's largest V block scale: each block's V scale rides in P;
+ *   - every block's P8 V8 is summed by the tensor core's fp32 accumulator
+ *     (fp32 accumulation across blocks); O = that sum * sV_max / 224 / l,
+ *     with the row sum l taken over the unquantised exponentials.
  *   q, k, v : in,  bf16 [B, S, H, D]
  *   o       : out, bf16 [B, S, H, D]
  *   lse     : out, fp32 [B, H, S], natural log, of the dequantised scores

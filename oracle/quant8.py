@@ -8,13 +8,16 @@ The pages' 8-bit FlashAttention: Wan 2.1 paper-podcast summary, section
 95% MFU on H20) and the kwkr.cn Wan explainer, section 4.2 (FlashAttention3
 8-bit: INT8 for Q, K, V, FP8 output, FP32 register accumulation).  The two
 disagree on which operands are int8; the reading taken here is int8 Q and K,
-e4m3 P and V, per-(batch, head, 64-token block) absmax scales, with every
-64-key block's P.V product taken out in fp32 and scaled there.
+e4m3 P and V, per-(batch, head, 64-token block) scales (absmax/127 for int8;
+for V the smallest power of two >= absmax/448), each block's V scale folded
+into P before P is quantised (an exact power-of-two factor), and all blocks'
+P.V products summed by one fp32 accumulation.
 
 Where a floating-point value decides a code (the scale, the quotient x/scale
 and its rounding), the computation is done in fp32 exactly as the CUDA
 quantiser does it, so codes can be compared bit for bit:
-    scale = fp32(absmax / 127)   (int8)     scale = fp32(absmax / 448)  (e4m3)
+    scale = fp32(absmax / 127)   (int8)
+    scale = max(smallest power of two >= fp32(absmax / 448), 2^-126)   (e4m3)
     scale = 1 when absmax == 0
     int8 code = clamp(rint_even(fp32(x / scale)), -127, 127)
     e4m3 code = e4m3_rne_satfinite(fp32(x / scale))
@@ -89,11 +92,23 @@ def quant_int8(x, block: int = BLOCK):
     return codes, scale
 
 
+def pow2_ceil_f32(q: np.ndarray) -> np.ndarray:
+    """The smallest power of two >= q (q > 0, fp32), exactly: q itself when q is one."""
+    mant, ex = np.frexp(q.astype(np.float32))            # q = mant * 2^ex, mant in [0.5, 1)
+    return np.where(mant == 0.5, q, np.ldexp(np.float32(1.0), ex)).astype(np.float32)
+
+
 def quant_e4m3(x, block: int = BLOCK):
-    """E4M3 codes (uint8 bit patterns) [B, S, H, D], their values (fp64) and fp32 scales [B, H, nblk] of V."""
+    """E4M3 codes (uint8 bit patterns) [B, S, H, D], their values (fp64) and fp32 scales [B, H, nblk] of V.
+
+    Each block's scale is the smallest power of two >= fp32(absmax / 448), at
+    least 2^-126 (1 for an all-zero block): the codes then span up to 448 and any
+    two blocks' scales differ by an exact power of two."""
     xf = _f32(x)
     amax = block_absmax(xf, block)
-    scale = np.where(amax == 0, np.float32(1.0), amax / np.float32(E4M3_MAX)).astype(np.float32)
+    q = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    scale = np.where(amax == 0, np.float32(1.0), pow2_ceil_f32(np.where(amax == 0, np.float32(1.0), q)))
+    scale = np.maximum(scale, np.float32(2.0 ** -126)).astype(np.float32)   # always a normal float
     per_tok = np.repeat(scale, block, axis=2)[:, :, : xf.shape[1]]
     quot = (xf / per_tok.transpose(0, 2, 1)[:, :, :, None]).astype(np.float32)
     return e4m3_bits(quot), e4m3_round(quot), scale
@@ -103,16 +118,17 @@ def attn_fwd_q8_sim(q, k, v, rows=None, heads=None, block: int = BLOCK):
     """Diagnostic fp64 simulation of the 8-bit recipe (not a parity gate).
 
     Scores from the int8 codes, s_ij = (q8_i . k8_j) sQ(i) sK(j) / sqrt(D);
-    p_ij = exp(s_ij - max_j s_ij) in [0, 1]; l_i = sum_j p_ij (unquantised);
-    P8 = e4m3(448 p); o_i = sum over 64-key blocks t of
-    (sum_{j in t} P8_ij v8_j) * sV(t) / 448, divided by l_i."""
+    p_ij = exp(s_ij - max_j s_ij) in [0, 1]; l_i = sum_j p_ij (unquantised).
+    Each 64-key block t's V scale is folded into P before P is quantised,
+    P8_ij = e4m3(448 p_ij sV(t) / sV_max) with sV_max the largest block scale
+    of the (b, h), so one fp32 accumulation carries every block:
+    o_i = (sum_j P8_ij v8_j) * sV_max / 448 / l_i."""
     B, S, H, D = q.shape
     rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
     heads = list(range(H)) if heads is None else list(heads)
     q8, sq = quant_int8(q, block)
     k8, sk = quant_int8(k, block)
     _, v8, sv = quant_e4m3(v, block)
-    nb = sk.shape[2]
     o = np.empty((B, len(rows), len(heads), D))
     lse = np.empty((B, len(heads), len(rows)))
     for b in range(B):
@@ -123,12 +139,10 @@ def attn_fwd_q8_sim(q, k, v, rows=None, heads=None, block: int = BLOCK):
             m = s.max(axis=1)
             p = np.exp(s - m[:, None])
             l = p.sum(axis=1)
-            p8 = e4m3_round(p * E4M3_MAX)
-            acc = np.zeros((len(rows), D))
-            for t in range(nb):
-                j0, j1 = t * block, min(S, (t + 1) * block)
-                acc += (p8[:, j0:j1] @ v8[b, j0:j1, h, :]) * (float(sv[b, h, t]) / E4M3_MAX)
-            o[b, :, hi, :] = acc / l[:, None]
+            sv_key = np.repeat(sv[b, h], block)[:S].astype(np.float64)        # sV of each key's block
+            sv_max = float(sv[b, h].max())
+            p8 = e4m3_round(p * (E4M3_MAX * sv_key / sv_max)[None, :])
+            o[b, :, hi, :] = (p8 @ v8[b, :, h, :]) * (sv_max / E4M3_MAX) / l[:, None]
             lse[b, hi] = m + np.log(l)
     return o, lse
 

@@ -69,7 +69,12 @@ def test_e4m3_block_quantisation():
     x = rng.standard_normal((1, 100, 2, 16)).astype(np.float32)
     bits, vals, scale = q8.quant_e4m3(x)
     amax = np.abs(x[:, :64]).max(axis=(1, 3))
-    np.testing.assert_array_equal(scale[:, :, 0], (amax / np.float32(448)).astype(np.float32))
+    # power-of-two scales: 2^k with 2^(k-1) < absmax/448 <= 2^k
+    s0 = scale[:, :, 0].astype(np.float64)
+    assert np.all(np.log2(s0) == np.round(np.log2(s0)))
+    assert np.all(s0 >= amax / 448.0) and np.all(s0 / 2 < amax / 448.0)
+    np.testing.assert_array_equal(q8.pow2_ceil_f32(np.float32([0.25, 0.3, 1.0, 3e-41, 5.0])),
+                                  np.float32([0.25, 0.5, 1.0, 2.0 ** -134, 8.0]))
     deq = vals * np.repeat(scale, 64, axis=2)[:, :, :100].transpose(0, 2, 1)[:, :, :, None]
     rel = np.abs(deq - x) / np.maximum(np.abs(x), 1e-3)
     assert np.percentile(rel, 99) < 0.07

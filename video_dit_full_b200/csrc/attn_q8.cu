@@ -3,24 +3,24 @@
 // The pages' 8-bit FlashAttention ("Wan 2.1 ... paper-podcast summary",
 // section "干预与形式化": mixed int8/FP8 with FP32 accumulation across blocks;
 // kwkr.cn Wan explainer, section 4.2 "FlashAttention3的8-bit优化"), read as:
-// int8 Q and K and e4m3 V with per-(batch, head, 64-token block) absmax scales,
-// P quantised to e4m3 as e4m3(448 p), and each 64-key block's P V product taken
-// out of the tensor core and added in fp32 with that block's V scale.
+// int8 Q and K with per-(batch, head, 64-token block) absmax/127 scales and e4m3 V
+// with per-block power-of-two scales (the smallest 2^k >= absmax/448);
+// P quantised to e4m3 with each 64-key block's V scale folded in,
+// P8 = e4m3(P_SCALE p sV_block / sV_max); every block's P8 V8 product summed by
+// the tensor core's fp32 accumulator; O = that sum * sV_max / P_SCALE / l.
 //
 // Two kernels:
 //   q8_quantize   one CTA per (tensor, b, h, 64-token block): absmax, scale,
 //                 codes (IEEE division, round to nearest even), written
 //                 head-major [B, H, S, 128] into the workspace.
-//   q8_attn       one CTA per 128-row Q tile of one (b, h), 128-key K/V tiles:
-//                 warp 16 TMA, warp 17 tcgen05 issuer, warps 0-7 softmax (two threads
-//                 per row, one 64-key block each, partial maxima swapped through
-//                 shared memory), warps 8-15 fp32 accumulation of O (two per row).
-//                   S = Q8 K8^T          kind::i8, int32 in TMEM (two buffers)
+//   q8_attn       one CTA per pair of 128-row Q tiles of one (b, h), sharing
+//                 128-key K8/V8 tiles (three-stage TMA rings); the same ping-pong
+//                 as the bf16 forward:
+//                   S_t = Q8_t K8^T         kind::i8, int32 in TMEM
 //                   s = S sQ sK / sqrt(D) * log2(e) per 64-key column block
-//                   P8 = e4m3(2^(s - m + log2 448)) -> TMEM (over S)
-//                   Ob_a, Ob_b = P8 V8 for the tile's two 64-key blocks (kind::f8f6f4)
-//                   O = O * 2^(m_old - m) + Ob_a sV_a + Ob_b sV_b   (fp32, registers)
-//                 The 448 of P cancels against l = sum 448 p in the epilogue.
+//                   P8_t = e4m3(2^(s - m + log2(P_SCALE sV_blk / sV_max)))  -> TMEM (over S_t)
+//                   O_t += P8_t V8        kind::f8f6f4, fp32 accumulator in TMEM
+//                 warp 8 TMA, warp 9 MMA, warps 0-3 / 4-7 softmax of Q tile 0 / 1.
 #include <cuda.h>
 
 #include "sm100_ptx.cuh"
@@ -80,8 +80,20 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const Q8QuantParams p)
     amax = warp_max[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
-    const float qmax = which == 2 ? 448.f : 127.f;
-    const float scale = amax > 0.f ? __fdiv_rn(amax, qmax) : 1.f;
+    float scale = 1.f;
+    if (amax > 0.f) {
+        if (which < 2) {
+            scale = __fdiv_rn(amax, 127.f);                   // int8: absmax / 127
+        } else {
+            // e4m3: the smallest power of two >= absmax / 448, so that the ratio of any two
+            // of a head's V block scales is an exact power of two (it is folded into P)
+            // (at least 2^-126, so every scale is a normal float whose exponent field gives k)
+            const float q = __fdiv_rn(amax, 448.f);
+            int e;
+            const float mant = frexpf(q, &e);                 // q = mant * 2^e, mant in [0.5, 1)
+            scale = fmaxf((mant == 0.5f) ? q : ldexpf(1.f, e), 0x1p-126f);
+        }
+    }
     const size_t out_off = ((static_cast<size_t>(bh) * p.S) + tok) * HD + part * 32;
     if (threadIdx.x == 0) {
         float* sc = which == 0 ? p.sq : which == 1 ? p.sk : p.sv;
@@ -118,35 +130,30 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const Q8QuantParams p)
     }
 }
 
-constexpr int BM = 128;                     // Q rows per CTA
+constexpr int BM = 128;                     // query rows per Q tile
 constexpr int BN = 128;                     // keys per K/V tile (two quantisation blocks)
+constexpr int NQ = 2;                       // Q tiles per CTA (they share every K/V tile)
 constexpr int T8 = BM * HD;                 // 16 KB 8-bit tile
 constexpr int STAGES = 3;
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + T8;
+constexpr int OFF_K = OFF_Q + NQ * T8;
 constexpr int OFF_V = OFF_K + STAGES * T8;
-constexpr int OFF_ALPHA = OFF_V + STAGES * T8;        // 4 x 128 fp32 rescale factors
-constexpr int OFF_STAT = OFF_ALPHA + 4 * BM * 4;      // final m per row, l per (half, row)
-constexpr int OFF_XMAX = OFF_STAT + 3 * BM * 4;       // [parity][half][row] partial row maxima
-constexpr int OFF_BAR = OFF_XMAX + 2 * 2 * BM * 4;
-enum Bar { Q_FULL = 0, K_FULL = 1, K_EMPTY = 4, V_FULL = 7, V_EMPTY = 10, S_FULL = 13, P_READY = 15,
-           ALPHA_READY = 17, OB_FULL = 21, OB_FREE = 22, STATS = 23, DRAIN = 24, XCHG = 25, NBARS = 27 };
+constexpr int OFF_RED = OFF_V + STAGES * T8;          // 16 floats: per-warp partial maxima of sV
+constexpr int OFF_BAR = OFF_RED + 64;
+enum Bar { Q_FULL = 0, K_FULL = 2, K_EMPTY = 5, V_FULL = 8, V_EMPTY = 11, S_FULL = 14, P_FULL = 16,
+           O_FINAL = 18, DRAIN = 20, NBARS = 21 };
 constexpr int OFF_TMEM_SLOT = OFF_BAR + NBARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
 constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
-// warps 0-7 softmax (two threads per row: warps 0-3 keys 0-63 of a tile = one quantisation
-// block, warps 4-7 keys 64-127), warps 8-15 fp32 accumulation of O (two threads per row:
-// d 0-63 / 64-127), 16 TMA, 17 MMA
-constexpr int NTHREADS = 576;
-constexpr int WARP_TMA = 16, WARP_MMA = 17;
-constexpr int HALF_THREADS = 256;
-#ifndef WAN_Q8_POLY_PAIRS
-#define WAN_Q8_POLY_PAIRS 0            // of every 8 pairs of exponentials, this many use exp2_poly3
-#endif
-constexpr int Q8_POLY_PAIRS = WAN_Q8_POLY_PAIRS;
-constexpr uint32_t TMEM_COLS = 512;         // S0 | S1 (int32, P8 over the first 32 columns) | Ob_a | Ob_b
-constexpr uint32_t T_OBA = 256, T_OBB = 384;
+constexpr int NTHREADS = 320;               // warps 0-3 softmax of Q tile 0, 4-7 of Q tile 1, 8 TMA, 9 MMA
+constexpr uint32_t TMEM_COLS = 512;         // S0 | S1 (int32; P8 over their first 32 columns) | O0 | O1
+constexpr uint32_t T_O = 256;
 constexpr float LOG2_448 = 8.807354922057604f;
+// The running max is moved only when it rises by more than 1 (log2 units), so p <= 2 against
+// the max in use; P is then quantised as e4m3(P_SCALE * p * sV_block / sV_max) <= 448.
+constexpr float RESCALE_THRESHOLD = 1.0f;
+constexpr float P_SCALE = 224.f;
+constexpr float LOG2_P_SCALE = 7.807354922057604f;
 
 // S (int32) = Q8 K8^T: both [128 rows][128 bytes] K-major with the 128-byte swizzle, K = 32 per MMA.
 __device__ __forceinline__ void issue_qk8(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem, uint32_t idesc) {
@@ -156,17 +163,15 @@ __device__ __forceinline__ void issue_qk8(uint32_t d_tmem, uint32_t q_smem, uint
                   idesc, kk > 0 ? 1u : 0u);
 }
 
-// Ob_a, Ob_b = P8 V8 for keys 0-63 and 64-127 of the tile; P8 in TMEM (4 per column; keys
-// 0-63 at columns 0-15, keys 64-127 at columns 64-79, each written by the thread that read them),
-// V8 [key][d] MN-major (one 128-byte swizzle atom spans all 128 d), 32 keys per MMA.
-__device__ __forceinline__ void issue_pv8(uint32_t tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc) {
+// O (fp32, TMEM) += P8 V8: P8 in TMEM (4 e4m3 per column, columns 0-31), V8 [key][d] MN-major
+// (one 128-byte swizzle atom spans all 128 d), 32 keys per MMA.  The tensor core's fp32
+// accumulator carries the sum across every 64-key block; each block's V scale is already in P8.
+__device__ __forceinline__ void issue_pv8(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc,
+                                          bool accumulate) {
 #pragma unroll
-    for (int a = 0; a < 2; ++a) {
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk)
-            mma_f8_ts(tmem + (a ? T_OBB : T_OBA), p_tmem + a * 64 + kk * 8,
-                      sdesc_sw128(v_smem + a * 8192 + kk * 4096, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-    }
+    for (int kk = 0; kk < BN / 32; ++kk)
+        mma_f8_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(v_smem + kk * 4096, 16, 1024), idesc,
+                  (accumulate || kk > 0) ? 1u : 0u);
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -181,41 +186,46 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     const int lane = lane_id();
     const int h = blockIdx.y, b = blockIdx.z;
     const int bh = b * p.H + h;
-    const int q0 = blockIdx.x * BM;
+    const int q0 = blockIdx.x * (NQ * BM);
     const int S = p.S;
+    const int nq = (q0 + BM < S) ? 2 : 1;
     const int nkv = (S + BN - 1) / BN;
 
     const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sV = base + OFF_V;
-    float* alpha_buf = reinterpret_cast<float*>(smem + OFF_ALPHA);
-    float* stat_m = reinterpret_cast<float*>(smem + OFF_STAT);
-    float* stat_l = stat_m + BM;                           // [half][row]
+    float* red = reinterpret_cast<float*>(smem + OFF_RED);
     const uint32_t bar0 = base + OFF_BAR;
     auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
     const WaitCtl wc{abort_flag, p.wait_budget_ns, p.status};
 
+    // sV_max of this (b, h): every thread folds a strided share, warps reduce by shuffle
+    const float* sv = p.sv + static_cast<size_t>(bh) * p.nblk;
+    {
+        float mv = 0.f;
+        for (int i = threadIdx.x; i < p.nblk; i += NTHREADS) mv = fmaxf(mv, sv[i]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, off));
+        if (lane == 0) red[warp] = mv;
+    }
     if (threadIdx.x == 0) {
         mbar_init(bar(Q_FULL), 1);
+        mbar_init(bar(Q_FULL + 1), 1);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar(K_FULL + s), 1);
             mbar_init(bar(K_EMPTY + s), 1);
             mbar_init(bar(V_FULL + s), 1);
             mbar_init(bar(V_EMPTY + s), 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(S_FULL + s), 1);
-            mbar_init(bar(P_READY + s), HALF_THREADS);
-            mbar_init(bar(XCHG + s), HALF_THREADS);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar(S_FULL + t), 1);
+            mbar_init(bar(P_FULL + t), BM);
+            mbar_init(bar(O_FINAL + t), 1);
         }
-        for (int s = 0; s < 4; ++s) mbar_init(bar(ALPHA_READY + s), HALF_THREADS);
-        mbar_init(bar(OB_FULL), 1);
-        mbar_init(bar(OB_FREE), HALF_THREADS);
-        mbar_init(bar(STATS), HALF_THREADS);
         mbar_init(bar(DRAIN), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == WARP_MMA) {
+    if (warp == 9) {
         tmem_alloc(base + OFF_TMEM_SLOT, TMEM_COLS);
         tmem_relinquish();
     }
@@ -223,15 +233,20 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
+    float sv_max = red[0];
+#pragma unroll
+    for (int w = 1; w < NTHREADS / 32; ++w) sv_max = fmaxf(sv_max, red[w]);
 
-    if (warp == WARP_TMA) {
+    if (warp == 8) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
             tma_prefetch_desc(&tmq);
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
-            mbar_arrive_expect_tx(bar(Q_FULL), T8);
-            tma_load_3d(sQ, &tmq, bar(Q_FULL), 0, q0, bh);
+            for (int t = 0; t < nq; ++t) {
+                mbar_arrive_expect_tx(bar(Q_FULL + t), T8);
+                tma_load_3d(sQ + t * T8, &tmq, bar(Q_FULL + t), 0, q0 + t * BM, bh);
+            }
             int kpar[STAGES], vpar[STAGES];
             for (int s = 0; s < STAGES; ++s) kpar[s] = vpar[s] = -1;
             bool ok = true;
@@ -250,190 +265,181 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 vpar[s] = use;
             }
             if (!ok) {
-                drain_wait(bar(Q_FULL), 0);
+                for (int t = 0; t < nq; ++t) drain_wait(bar(Q_FULL + t), 0);
                 for (int s = 0; s < STAGES; ++s) {
                     if (kpar[s] >= 0) drain_wait(bar(K_FULL + s), kpar[s]);
                     if (vpar[s] >= 0) drain_wait(bar(V_FULL + s), vpar[s]);
                 }
             }
         }
-    } else if (warp == WARP_MMA) {
+    } else if (warp == 9) {
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
             const uint32_t idesc_qk = make_idesc(2, 1, 1, 0, 0, BM, BN);   // s32 <- s8 x s8
             const uint32_t idesc_pv = make_idesc(1, 0, 0, 0, 1, BM, HD);   // f32 <- e4m3 x e4m3, V MN-major
-            bool ok = wait_thread(bar(Q_FULL), 0, wc);
-            for (int j = 0; j < 2 && j < nkv && ok; ++j) {
-                ok = wait_thread(bar(K_FULL + j), 0, wc);
-                if (!ok) break;
+            bool ok = true;
+            for (int t = 0; t < nq && ok; ++t) ok = wait_thread(bar(Q_FULL + t), 0, wc);
+            if (ok) ok = wait_thread(bar(K_FULL + 0), 0, wc);
+            if (ok) {
                 tc_fence_after();
-                issue_qk8(tmem + j * BN, sQ, sK + j * T8, idesc_qk);
-                mma_commit(bar(S_FULL + j));
-                mma_commit(bar(K_EMPTY + j));
+                for (int t = 0; t < nq; ++t) {
+                    issue_qk8(tmem + t * BN, sQ + t * T8, sK, idesc_qk);
+                    mma_commit(bar(S_FULL + t));
+                }
+                mma_commit(bar(K_EMPTY + 0));
             }
             for (int j = 0; j < nkv && ok; ++j) {
-                const int sb = j & 1;
-                const int vs = j % STAGES;
-                ok = wait_thread(bar(P_READY + sb), (j >> 1) & 1, wc);
-                if (ok && j > 0) ok = wait_thread(bar(OB_FREE), (j - 1) & 1, wc);
-                if (ok) ok = wait_thread(bar(V_FULL + vs), (j / STAGES) & 1, wc);
-                if (!ok) break;
-                tc_fence_after();
-                issue_pv8(tmem, tmem + sb * BN, sV + vs * T8, idesc_pv);
-                mma_commit(bar(OB_FULL));
-                mma_commit(bar(V_EMPTY + vs));
-                if (j + 2 < nkv) {
-                    const int ks = (j + 2) % STAGES;
-                    ok = wait_thread(bar(K_FULL + ks), ((j + 2) / STAGES) & 1, wc);
+                const int s = j % STAGES;
+                const int s1 = (j + 1) % STAGES;
+                ok = wait_thread(bar(V_FULL + s), (j / STAGES) & 1, wc);
+                for (int t = 0; t < nq && ok; ++t) {
+                    ok = wait_thread(bar(P_FULL + t), j & 1, wc);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_qk8(tmem + sb * BN, sQ, sK + ks * T8, idesc_qk);   // after P V read this buffer
-                    mma_commit(bar(S_FULL + sb));
-                    mma_commit(bar(K_EMPTY + ks));
+                    issue_pv8(tmem + T_O + t * HD, tmem + t * BN, sV + s * T8, idesc_pv, j > 0);
+                    if (j + 1 == nkv) mma_commit(bar(O_FINAL + t));
+                    if (j + 1 < nkv) {
+                        if (t == 0) {
+                            ok = wait_thread(bar(K_FULL + s1), ((j + 1) / STAGES) & 1, wc);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                        issue_qk8(tmem + t * BN, sQ + t * T8, sK + s1 * T8, idesc_qk);   // after P V read it
+                        mma_commit(bar(S_FULL + t));
+                    }
                 }
+                if (!ok) break;
+                mma_commit(bar(V_EMPTY + s));
+                if (j + 1 < nkv) mma_commit(bar(K_EMPTY + s1));
             }
             mma_commit(bar(DRAIN));
             drain_wait(bar(DRAIN), 0);
         }
-    } else if (warp < 8) {
-        // ------------------- softmax (row r, key half hc = one 64-key block) -------
-        const int hc = warp >> 2;
-        const int r = (warp & 3) * 32 + lane;
+    } else {
+        // ---------------- softmax, O rescale and epilogue (row r of Q tile t) ------------
+        const int t = warp >> 2;
+        const int r = threadIdx.x & 127;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const int row = q0 + r;
+        const uint32_t tS = tmem + t * BN + lane_off;
+        const uint32_t tO = tmem + T_O + t * HD + lane_off;
+        const int row = q0 + t * BM + r;
         const float* sk = p.sk + static_cast<size_t>(bh) * p.nblk;
         const float sq_row = p.sq[static_cast<size_t>(bh) * p.nblk + min(row, S - 1) / BLK];
-        float* xmax = reinterpret_cast<float*>(smem + OFF_XMAX);
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
+        const int sv_max_exp = static_cast<int>(__float_as_uint(sv_max) >> 23);   // positive, normal
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = (t < nq);
         for (int j = 0; j < nkv && ok; ++j) {
-            const int sb = j & 1;
-            const int kb = 2 * j + hc;                      // this thread's quantisation block
-            ok = wait_warp(bar(S_FULL + sb), (j >> 1) & 1, wc);
+            ok = wait_warp(bar(S_FULL + t), j & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tS = tmem + sb * BN + lane_off + hc * 64;
-            uint32_t sr[64];
-            tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            uint32_t sr[128];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q * 32]));
             tmem_wait_ld();
-            const float cs = kb < p.nblk ? sq_row * sk[kb] * p.scale_log2 : 0.f;
+            const int kb = 2 * j;
+            const bool has_b = kb + 1 < p.nblk;
+            const float ca = sq_row * sk[kb] * p.scale_log2;
+            const float cb = has_b ? sq_row * sk[kb + 1] * p.scale_log2 : 0.f;
             float* s = reinterpret_cast<float*>(sr);
-            // int32 -> fp32 without the conversion unit: |S| <= 128*127*127 < 2^22, so
-            // adding 1.5*2^23 as a float bit pattern and subtracting it back is exact.
+            // int32 -> fp32 without the conversion unit: |S| <= 128*127*127 < 2^22, so adding
+            // 1.5*2^23 as a float bit pattern and subtracting it back is exact.
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-                s[c] = (__int_as_float(static_cast<int>(sr[c]) + 0x4B400000) - 12582912.f) * cs;
-            const int valid = S - j * BN - hc * 64;
-            if (valid < 64) {
+            for (int c = 0; c < 128; ++c)
+                s[c] = (__int_as_float(static_cast<int>(sr[c]) + 0x4B400000) - 12582912.f) * (c < 64 ? ca : cb);
+            const int valid = S - j * BN;
+            if (valid < BN) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
+                for (int c = 0; c < 128; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
             float m8[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) m8[c] = s[c];
 #pragma unroll
-            for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+            for (int c = 8; c < 128; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
 #pragma unroll
             for (int w = 4; w > 0; w >>= 1)
 #pragma unroll
                 for (int c = 0; c < w; ++c) m8[c] = fmaxf(m8[c], m8[c + w]);
-            // swap partial maxima with the other half of the row
-            const int xb = (sb * 2) * BM;
-            xmax[xb + hc * BM + r] = m8[0];
-            mbar_arrive(bar(XCHG + sb));
-            ok = wait_warp(bar(XCHG + sb), (j >> 1) & 1, wc);
-            if (!ok) break;
-            const float mx = fmaxf(m8[0], xmax[xb + (hc ^ 1) * BM + r]);
-            const float m_new = fmaxf(m, mx);
-            const float alpha = ex2_approx(m - m_new);
-            const float bias = m_new - LOG2_448;       // p * 448 = 2^(s - bias) <= 448
-            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[16];
+            float alpha = 1.f;
+            bool moved = false;
+            if (m8[0] > m_ref + RESCALE_THRESHOLD) {
+                alpha = ex2_approx(m_ref - m8[0]);
+                m_ref = m8[0];
+                moved = true;
+            }
+            // P_SCALE * p * sV_blk / sV_max = 2^(s - m_ref + lg_blk), lg_blk = log2(P_SCALE * sV_blk / sV_max)
+            // V block scales are normal powers of two: r = sV_blk / sV_max = 2^-k exactly, k read off
+            // the exponent fields
+            // (k is clamped to 64: any block 2^-20 below the largest already quantises to zero)
+            const int ka = min(sv_max_exp - static_cast<int>(__float_as_uint(sv[kb]) >> 23), 64);
+            const int kbb = has_b ? min(sv_max_exp - static_cast<int>(__float_as_uint(sv[kb + 1]) >> 23), 64) : 0;
+            const float inv_a = __uint_as_float(static_cast<uint32_t>(127 + ka) << 23) * (1.f / P_SCALE);
+            const float inv_b = __uint_as_float(static_cast<uint32_t>(127 + kbb) << 23) * (1.f / P_SCALE);
+            const float ba = m_ref - (LOG2_P_SCALE - static_cast<float>(ka));
+            const float bbias = m_ref - (LOG2_P_SCALE - static_cast<float>(kbb));
+            float sa4[4] = {0.f, 0.f, 0.f, 0.f}, sb4[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[32];
 #pragma unroll
-            for (int w = 0; w < 16; ++w) {
-                const bool poly = ((2 * w) & 7) < 2 * Q8_POLY_PAIRS;
-                const float x0 = s[4 * w] - bias, x1 = s[4 * w + 1] - bias;
-                const float x2 = s[4 * w + 2] - bias, x3 = s[4 * w + 3] - bias;
-                const float p0 = poly ? exp2_poly3(x0) : ex2_approx(x0);
-                const float p1 = poly ? exp2_poly3(x1) : ex2_approx(x1);
-                const float p2 = poly ? exp2_poly3(x2) : ex2_approx(x2);
-                const float p3 = poly ? exp2_poly3(x3) : ex2_approx(x3);
-                sum4[w & 3] += (p0 + p1) + (p2 + p3);
+            for (int w = 0; w < 32; ++w) {
+                const float bias = w < 16 ? ba : bbias;
+                const float p0 = ex2_approx(s[4 * w] - bias), p1 = ex2_approx(s[4 * w + 1] - bias);
+                const float p2 = ex2_approx(s[4 * w + 2] - bias), p3 = ex2_approx(s[4 * w + 3] - bias);
+                if (w < 16) sa4[w & 3] += (p0 + p1) + (p2 + p3);
+                else sb4[w & 3] += (p0 + p1) + (p2 + p3);
                 pk[w] = pack_e4m3x2(p0, p1) | (pack_e4m3x2(p2, p3) << 16);
             }
-            tmem_st16(tS, pk);                                 // P8 over the columns this thread read
-            l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
-            m = m_new;
-            if (hc == 0) alpha_buf[(j & 3) * BM + r] = alpha;
-            mbar_arrive(bar(ALPHA_READY + (j & 3)));
+            tmem_st32(tS, pk);                                   // P8 over S's first 32 columns
+            // the row sum counts p itself: scale each block's sum by 1 / (P_SCALE * r_blk) = 2^k / P_SCALE
+            const float sum = ((sa4[0] + sa4[1]) + (sa4[2] + sa4[3])) * inv_a +
+                              ((sb4[0] + sb4[1]) + (sb4[2] + sb4[3])) * inv_b;
+            l = l * alpha + sum;
+            if (j > 0 && __any_sync(0xffffffffu, moved)) {
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + q * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tO + q * 32, o);
+                }
+            }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(P_READY + sb));
+            mbar_arrive(bar(P_FULL + t));
         }
+        if (ok) ok = wait_warp(bar(O_FINAL + t), 0, wc);
         if (ok) {
-            if (hc == 0) stat_m[r] = m;
-            stat_l[hc * BM + r] = l;
-            mbar_arrive(bar(STATS));
-        }
-    } else {
-        // ------------- fp32 accumulation of O (row r, d half hd) -----------------
-        const int hd = (warp >> 2) & 1;
-        const int r = (warp & 3) * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const int row = q0 + r;
-        const float* sv = p.sv + static_cast<size_t>(bh) * p.nblk;
-        float o[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) o[c] = 0.f;
-        bool ok = true;
-        for (int j = 0; j < nkv && ok; ++j) {
-            ok = wait_warp(bar(ALPHA_READY + (j & 3)), (j >> 2) & 1, wc);
-            if (!ok) break;
-            const float alpha = alpha_buf[(j & 3) * BM + r];
-            ok = wait_warp(bar(OB_FULL), j & 1, wc);
-            if (!ok) break;
             tc_fence_after();
-            const int kb = 2 * j;
-            const float sva = sv[kb];
-            const float svb = kb + 1 < p.nblk ? sv[kb + 1] : 0.f;
-#pragma unroll
+            // O = (sum over blocks of P8 V8) * sV_max / P_SCALE / l
+            const float mul = sv_max / (P_SCALE * l);
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
+                                  ((static_cast<size_t>(b) * S + row) * p.H + h) * HD;
+#pragma unroll 1
             for (int q = 0; q < 4; ++q) {
-                uint32_t a[16], bb[16];
-                tmem_ld16(tmem + T_OBA + lane_off + hd * 64 + q * 16, a);
-                tmem_ld16(tmem + T_OBB + lane_off + hd * 64 + q * 16, bb);
+                uint32_t o[32];
+                tmem_ld32(tO + q * 32, o);
                 tmem_wait_ld();
+                uint4 pk4[4];
+                uint32_t* pw = reinterpret_cast<uint32_t*>(pk4);
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    o[q * 16 + e] = fmaf(__uint_as_float(a[e]), sva,
-                                         fmaf(__uint_as_float(bb[e]), svb, o[q * 16 + e] * alpha));
-            }
-            tc_fence_before();
-            mbar_arrive(bar(OB_FREE));
-        }
-        if (ok) ok = wait_warp(bar(STATS), 0, wc);
-        if (ok && row < S) {
-            const float m = stat_m[r], l = stat_l[r] + stat_l[BM + r];
-            const float inv_l = 1.f / l;
-            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                  ((static_cast<size_t>(b) * S + row) * p.H + h) * HD + hd * 64;
-            uint4* d4 = reinterpret_cast<uint4*>(orow);
+                    pw[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
+                if (row < S) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                d4[u] = make_uint4(pack_bf16x2(o[8 * u] * inv_l, o[8 * u + 1] * inv_l),
-                                   pack_bf16x2(o[8 * u + 2] * inv_l, o[8 * u + 3] * inv_l),
-                                   pack_bf16x2(o[8 * u + 4] * inv_l, o[8 * u + 5] * inv_l),
-                                   pack_bf16x2(o[8 * u + 6] * inv_l, o[8 * u + 7] * inv_l));
-            if (hd == 0)
-                p.lse[static_cast<size_t>(bh) * S + row] = (m + log2f(l) - LOG2_448) * 0.69314718055994531f;
+                    for (int e = 0; e < 4; ++e) dst[e] = pk4[e];
+                }
+            }
+            if (row < S) p.lse[static_cast<size_t>(bh) * S + row] = (m_ref + log2f(l)) * 0.69314718055994531f;
         }
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == WARP_MMA) tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == 9) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 }  // namespace q8
@@ -444,7 +450,7 @@ int launch_q8(const Q8QuantParams& qp, const CUtensorMap& tq8, const CUtensorMap
     q8::q8_quantize_kernel<<<static_cast<unsigned>(nq), 256, 0, stream>>>(qp);
     if (cudaGetLastError() != cudaSuccess) return -1;
     if (configure_smem(reinterpret_cast<const void*>(q8::q8_attn_kernel), q8::SMEM_BYTES) != 0) return -1;
-    const dim3 grid((p.S + q8::BM - 1) / q8::BM, p.H, p.B);
+    const dim3 grid((p.S + q8::NQ * q8::BM - 1) / (q8::NQ * q8::BM), p.H, p.B);
     q8::q8_attn_kernel<<<grid, q8::NTHREADS, q8::SMEM_BYTES, stream>>>(tq8, tk8, tv8, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
