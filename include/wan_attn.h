@@ -110,8 +110,9 @@ WAN_ATTN_API size_t wan_attn_fwd_q8_workspace_size(int B, int S, int H, int D);
  *   - per (b, h, 64-token block): sQ = absmax(Q)/127, sK = absmax(K)/127,
  *     sV = the smallest power of two >= absmax(V)/448, at least 2^-126
  *     (fp32; every scale is 1 for an all-zero block); codes
- *     Q8 = clamp(rint(q / sQ), -127, 127), K8 likewise, V8 = e4m3(v / sV),
- *     each division IEEE fp32, rounding to nearest even, e4m3 saturating;
+ *     Q8 = clamp(rint(q * fp32(127 / absmax(Q))), -127, 127) with an fp32
+ *     product, K8 likewise, V8 = e4m3(v / sV) (exact: sV is a power of two),
+ *     rounding to nearest even, e4m3 saturating;
  *   - scores S = (Q8 . K8) sQ sK / sqrt(D) from int32 tensor-core sums;
  *   - P8 = e4m3(224 * exp(S - m) * sV_block / sV_max), where m is the running
  *     row max (moved only when it rises by more than a factor 2) and sV_max

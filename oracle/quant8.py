@@ -13,14 +13,14 @@ for V the smallest power of two >= absmax/448), each block's V scale folded
 into P before P is quantised (an exact power-of-two factor), and all blocks'
 P.V products summed by one fp32 accumulation.
 
-Where a floating-point value decides a code (the scale, the quotient x/scale
-and its rounding), the computation is done in fp32 exactly as the CUDA
-quantiser does it, so codes can be compared bit for bit:
-    scale = fp32(absmax / 127)   (int8)
+Where a floating-point value decides a code (the scale, the scaled value and
+its rounding), the computation is done in fp32 exactly as the CUDA quantiser
+does it, so codes can be compared bit for bit:
+    scale = fp32(absmax / 127), codes from fp32(x * fp32(127 / absmax))   (int8)
     scale = max(smallest power of two >= fp32(absmax / 448), 2^-126)   (e4m3)
     scale = 1 when absmax == 0
-    int8 code = clamp(rint_even(fp32(x / scale)), -127, 127)
-    e4m3 code = e4m3_rne_satfinite(fp32(x / scale))
+    int8 code = clamp(rint_even(fp32(x * fp32(127 / absmax))), -127, 127)
+    e4m3 code = e4m3_rne_satfinite(x / scale)        (exact: scale is a power of two)
 
 The unquantised fp64 oracle (``oracle.attention.attn_fwd``) is what the 8-bit
 path's parity is judged against; ``attn_fwd_q8_sim`` is a diagnostic only.
@@ -82,12 +82,16 @@ def block_absmax(x: np.ndarray, block: int = BLOCK) -> np.ndarray:
 
 
 def quant_int8(x, block: int = BLOCK):
-    """int8 codes [B, S, H, D] and fp32 scales [B, H, nblk] of Q or K."""
+    """int8 codes [B, S, H, D] and fp32 scales [B, H, nblk] of Q or K.
+
+    scale = fp32(absmax / 127) dequantises; the codes are rint(fp32(x * fp32(127 / absmax)))."""
     xf = _f32(x)
     amax = block_absmax(xf, block)
     scale = np.where(amax == 0, np.float32(1.0), amax / np.float32(127.0)).astype(np.float32)
-    per_tok = np.repeat(scale, block, axis=2)[:, :, : xf.shape[1]]          # [B, H, S]
-    quot = (xf / per_tok.transpose(0, 2, 1)[:, :, :, None]).astype(np.float32)
+    safe = np.where(amax == 0, np.float32(1.0), amax).astype(np.float32)
+    inv = np.where(amax == 0, np.float32(1.0), np.float32(127.0) / safe).astype(np.float32)
+    per_tok = np.repeat(inv, block, axis=2)[:, :, : xf.shape[1]]            # [B, H, S]
+    quot = (xf * per_tok.transpose(0, 2, 1)[:, :, :, None]).astype(np.float32)
     codes = np.clip(np.rint(quot), -127, 127).astype(np.int8)
     return codes, scale
 

@@ -1,8 +1,8 @@
 """The 8-bit forward (wan_attn_fwd_q8, through the C ABI).
 
 * Quantisation codes and scales are integer/byte work decided in fp32 on both
-  sides: bit-exact against ``oracle.quant8`` (IEEE division, round to nearest
-  even, e4m3 saturating).
+  sides: bit-exact against ``oracle.quant8`` (fp32 products with the block's
+  reciprocal scale, round to nearest even, e4m3 saturating).
 * O against the UNQUANTISED fp64 oracle: relative Frobenius error <= 4e-2
   (the workload's bar).  The recipe's own error on N(0,1) inputs is ~3.9e-2
   (the fp64 simulation ``oracle.quant8.attn_fwd_q8_sim``), so the kernel must

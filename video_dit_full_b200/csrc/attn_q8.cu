@@ -11,7 +11,8 @@
 //
 // Two kernels:
 //   q8_quantize   one CTA per (tensor, b, h, 64-token block): absmax, scale,
-//                 codes (IEEE division, round to nearest even), written
+//                 codes (fp32 products with the block's reciprocal scale, round to
+//                 nearest even), written
 //                 head-major [B, H, S, 128] into the workspace.
 //   q8_attn       one CTA per pair of 128-row Q tiles of one (b, h), sharing
 //                 128-key K8/V8 tiles (three-stage TMA rings); the same ping-pong
@@ -80,10 +81,11 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const Q8QuantParams p)
     amax = warp_max[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
-    float scale = 1.f;
+    float scale = 1.f, inv = 1.f;                          // codes = x * inv
     if (amax > 0.f) {
         if (which < 2) {
-            scale = __fdiv_rn(amax, 127.f);                   // int8: absmax / 127
+            scale = __fdiv_rn(amax, 127.f);                   // int8: dequantisation scale absmax / 127
+            inv = __fdiv_rn(127.f, amax);                     // one division per block, then products
         } else {
             // e4m3: the smallest power of two >= absmax / 448, so that the ratio of any two
             // of a head's V block scales is an exact power of two (it is folded into P)
@@ -92,6 +94,7 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const Q8QuantParams p)
             int e;
             const float mant = frexpf(q, &e);                 // q = mant * 2^e, mant in [0.5, 1)
             scale = fmaxf((mant == 0.5f) ? q : ldexpf(1.f, e), 0x1p-126f);
+            inv = 1.f / scale;                                // exact: scale is a power of two
         }
     }
     const size_t out_off = ((static_cast<size_t>(bh) * p.S) + tok) * HD + part * 32;
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const Q8QuantParams p)
             uint32_t word = 0;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                float c = rintf(__fdiv_rn(x[u * 4 + e], scale));
+                float c = rintf(__fmul_rn(x[u * 4 + e], inv));
                 c = fminf(fmaxf(c, -127.f), 127.f);
                 word |= (static_cast<uint32_t>(static_cast<int>(c)) & 0xFFu) << (8 * e);
             }
@@ -120,8 +123,8 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const Q8QuantParams p)
     } else {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const uint32_t lo = pack_e4m3x2(__fdiv_rn(x[u * 4], scale), __fdiv_rn(x[u * 4 + 1], scale));
-            const uint32_t hi = pack_e4m3x2(__fdiv_rn(x[u * 4 + 2], scale), __fdiv_rn(x[u * 4 + 3], scale));
+            const uint32_t lo = pack_e4m3x2(__fmul_rn(x[u * 4], inv), __fmul_rn(x[u * 4 + 1], inv));
+            const uint32_t hi = pack_e4m3x2(__fmul_rn(x[u * 4 + 2], inv), __fmul_rn(x[u * 4 + 3], inv));
             w[u] = lo | (hi << 16);
         }
         uint4* d4 = reinterpret_cast<uint4*>(p.v8 + out_off);
