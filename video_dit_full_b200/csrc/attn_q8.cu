@@ -345,25 +345,36 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             const float cb = has_b ? sq_row * sk[kb + 1] * p.scale_log2 : 0.f;
             float* s = reinterpret_cast<float*>(sr);
             // int32 -> fp32 without the conversion unit: |S| <= 128*127*127 < 2^22, so adding
-            // 1.5*2^23 as a float bit pattern and subtracting it back is exact.
+            // 1.5*2^23 as a float bit pattern and subtracting it back is exact.  Pairs of scores
+            // go through packed fp32 instructions (FADD2 / FMUL2).
+            {
+                const float2 k2 = make_float2(-12582912.f, -12582912.f);
+                const float2 ca2 = make_float2(ca, ca), cb2 = make_float2(cb, cb);
 #pragma unroll
-            for (int c = 0; c < 128; ++c)
-                s[c] = (__int_as_float(static_cast<int>(sr[c]) + 0x4B400000) - 12582912.f) * (c < 64 ? ca : cb);
+                for (int c = 0; c < 128; c += 2) {
+                    const float2 xm = make_float2(__int_as_float(static_cast<int>(sr[c]) + 0x4B400000),
+                                                  __int_as_float(static_cast<int>(sr[c + 1]) + 0x4B400000));
+                    const float2 v = fmul2(fadd2(xm, k2), c < 64 ? ca2 : cb2);
+                    s[c] = v.x;
+                    s[c + 1] = v.y;
+                }
+            }
             const int valid = S - j * BN;
             if (valid < BN) {
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
+            // row max: 8 chains of three-input maxima, then a short tree
             float m8[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) m8[c] = s[c];
+            for (int q = 0; q < 8; ++q) m8[q] = fmax3(s[q], s[q + 8], s[q + 16]);
 #pragma unroll
-            for (int c = 8; c < 128; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+            for (int q = 24; q < 128; q += 16)
 #pragma unroll
-            for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-                for (int c = 0; c < w; ++c) m8[c] = fmaxf(m8[c], m8[c + w]);
+                for (int e = 0; e < 8; ++e) m8[e] = (q + 8 + e < 128) ? fmax3(m8[e], s[q + e], s[q + 8 + e])
+                                                                       : fmaxf(m8[e], s[q + e]);
+            m8[0] = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
             float alpha = 1.f;
             bool moved = false;
             if (m8[0] > m_ref + RESCALE_THRESHOLD) {
@@ -381,21 +392,25 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             const float inv_b = __uint_as_float(static_cast<uint32_t>(127 + kbb) << 23) * (1.f / P_SCALE);
             const float ba = m_ref - (LOG2_P_SCALE - static_cast<float>(ka));
             const float bbias = m_ref - (LOG2_P_SCALE - static_cast<float>(kbb));
-            float sa4[4] = {0.f, 0.f, 0.f, 0.f}, sb4[4] = {0.f, 0.f, 0.f, 0.f};
+            float2 sa2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            float2 sb2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            const float2 nba = make_float2(-ba, -ba), nbb = make_float2(-bbias, -bbias);
             uint32_t pk[32];
 #pragma unroll
             for (int w = 0; w < 32; ++w) {
-                const float bias = w < 16 ? ba : bbias;
-                const float p0 = ex2_approx(s[4 * w] - bias), p1 = ex2_approx(s[4 * w + 1] - bias);
-                const float p2 = ex2_approx(s[4 * w + 2] - bias), p3 = ex2_approx(s[4 * w + 3] - bias);
-                if (w < 16) sa4[w & 3] += (p0 + p1) + (p2 + p3);
-                else sb4[w & 3] += (p0 + p1) + (p2 + p3);
-                pk[w] = pack_e4m3x2(p0, p1) | (pack_e4m3x2(p2, p3) << 16);
+                const float2 nb = w < 16 ? nba : nbb;
+                const float2 x01 = fadd2(make_float2(s[4 * w], s[4 * w + 1]), nb);
+                const float2 x23 = fadd2(make_float2(s[4 * w + 2], s[4 * w + 3]), nb);
+                const float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+                const float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+                if (w < 16) sa2[w & 1] = fadd2(sa2[w & 1], fadd2(p01, p23));
+                else sb2[w & 1] = fadd2(sb2[w & 1], fadd2(p01, p23));
+                pk[w] = pack_e4m3x2(p01.x, p01.y) | (pack_e4m3x2(p23.x, p23.y) << 16);
             }
             tmem_st32(tS, pk);                                   // P8 over S's first 32 columns
             // the row sum counts p itself: scale each block's sum by 1 / (P_SCALE * r_blk) = 2^k / P_SCALE
-            const float sum = ((sa4[0] + sa4[1]) + (sa4[2] + sa4[3])) * inv_a +
-                              ((sb4[0] + sb4[1]) + (sb4[2] + sb4[3])) * inv_b;
+            const float sum = ((sa2[0].x + sa2[0].y) + (sa2[1].x + sa2[1].y)) * inv_a +
+                              ((sb2[0].x + sb2[0].y) + (sb2[1].x + sb2[1].y)) * inv_b;
             l = l * alpha + sum;
             if (j > 0 && __any_sync(0xffffffffu, moved)) {
 #pragma unroll 1
