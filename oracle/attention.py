@@ -12,12 +12,18 @@ What it computes, and where the pages fix it:
   C = L(a*b*s*h^2 + b*b*s^2*h), "non-causal attention, beta = 4 forward,
   8 backward") and section "干预与形式化" (the DiT uses full spatio-temporal
   self-attention, not windowed);  kwkr.cn Wan explainer, section 2.2.
+* The same definition with queries and keys of different lengths is the DiT
+  block's cross-attention from the video tokens to the 512-token umT5 text
+  embedding (Wan 2.1 paper-podcast summary, section "干预与形式化": c_txt is
+  umT5's 512-token text embedding; the DiT backbone injects umT5 by
+  cross-attention).  Q and dO hold Sq rows, K and V hold Sk rows; self-
+  attention is Sk = Sq.
 * The softmax scale 1/sqrt(D), D = 128, the [B, S, H, D] layout and the
   natural-log LSE [B, H, S] are readings (the pages give no formula); the
   design notes list them.
 
 For each batch b, head h and query row i (inputs widened exactly from bf16):
-    s_ij  = (q_i . k_j) / sqrt(D)             for every key j in [0, S)
+    s_ij  = (q_i . k_j) / sqrt(D)             for every key j in [0, Sk)
     lse_i = m_i + ln sum_j exp(s_ij - m_i),    m_i = max_j s_ij
     o_i   = sum_j exp(s_ij - lse_i) v_j
 
@@ -63,8 +69,8 @@ def _rows_fwd(Q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float):
 def attn_fwd(q, k, v, rows=None, heads=None):
     """Forward attention.
 
-    q, k, v: [B, S, H, D] arrays (bf16 bit patterns or floats).
-    rows: query token indices to evaluate (default: all S).
+    q: [B, Sq, H, D], k and v: [B, Sk, H, D] arrays (bf16 bit patterns or floats).
+    rows: query token indices to evaluate (default: all Sq).
     heads: head indices to evaluate (default: all H).
     Returns (o [B, R, Hs, D] fp64, lse [B, Hs, R] fp64).
     """
@@ -89,16 +95,18 @@ def attn_fwd(q, k, v, rows=None, heads=None):
 def attn_bwd(q, k, v, do, q_rows=None, k_rows=None, heads=None):
     """Backward attention of f = sum(O * dO).
 
-    q_rows: query rows whose dQ is wanted (default all; empty = none).
-    k_rows: key rows whose dK, dV are wanted (default all; empty = none).
+    q, do: [B, Sq, H, D]; k, v: [B, Sk, H, D].
+    q_rows: query rows whose dQ is wanted (default all Sq; empty = none).
+    k_rows: key rows whose dK, dV are wanted (default all Sk; empty = none).
     heads:  heads to evaluate (default all).
     Returns dict with dq [B, Rq, Hs, D], dk and dv [B, Rk, Hs, D], and the
-    forward's lse [B, Hs, S] and Dl = rowsum(dO * O) [B, Hs, S] when key rows
-    were asked for (they need every row), else for the query rows only.
+    forward's lse [B, Hs, Sq] and Dl = rowsum(dO * O) [B, Hs, Sq] when key rows
+    were asked for (they need every query row), else for the query rows only.
     """
     B, S, H, D = q.shape
+    Sk = k.shape[1]
     q_rows = np.arange(S) if q_rows is None else np.asarray(q_rows, dtype=np.int64)
-    k_rows = np.arange(S) if k_rows is None else np.asarray(k_rows, dtype=np.int64)
+    k_rows = np.arange(Sk) if k_rows is None else np.asarray(k_rows, dtype=np.int64)
     heads = list(range(H)) if heads is None else list(heads)
     scale = 1.0 / np.sqrt(D)
     Hs = len(heads)

@@ -148,6 +148,9 @@ def tokens_for_video(frames: int, height: int, width: int) -> int:
     return (1 + (frames - 1) // 4) * (height // 16) * (width // 16)
 
 
+TEXT_TOKENS = 512   # length of the umT5 text embedding the DiT cross-attends to
+
+
 @dataclass(frozen=True)
 class Workload:
     name: str
@@ -159,11 +162,20 @@ class Workload:
     peaky_frac: float = 0.0        # fraction of heads whose Q is scaled x2
     backward: bool = False
     q8: bool = False
+    Skv: int | None = None         # key/value tokens when they differ from S (cross-attention)
+
+    @property
+    def kv_len(self) -> int:
+        return self.S if self.Skv is None else self.Skv
+
+    @property
+    def cross(self) -> bool:
+        return self.Skv is not None
 
     @property
     def fwd_flop(self) -> float:
-        """4*B*H*S^2*D: the forward's two S x S x D contractions (multiply-add = 2)."""
-        return 4.0 * self.B * self.H * self.S * self.S * self.D
+        """4*B*H*S*Skv*D: the forward's two S x Skv x D contractions (multiply-add = 2)."""
+        return 4.0 * self.B * self.H * self.S * self.kv_len * self.D
 
 
 WORKLOADS = {
@@ -177,6 +189,12 @@ WORKLOADS = {
                                    video=(81, 480, 832), backward=True),
     "q8_720p": Workload("q8_720p", 1, tokens_for_video(81, 720, 1280), 40, 128,
                         video=(81, 720, 1280), q8=True),
+    # the DiT block's cross-attention: video-token queries against the 512-token umT5 text
+    # embedding (Wan 2.1 paper-podcast summary, section "干预与形式化")
+    "cross_720p": Workload("cross_720p", 1, tokens_for_video(81, 720, 1280), 40, 128,
+                           video=(81, 720, 1280), Skv=TEXT_TOKENS),
+    "cross_train_480p": Workload("cross_train_480p", 1, tokens_for_video(81, 480, 832), 40, 128,
+                                 video=(81, 480, 832), backward=True, Skv=TEXT_TOKENS),
 }
 
 
@@ -206,15 +224,19 @@ def make_tensor(shape, seed: int, stream: int, nthreads=None) -> np.ndarray:
 
 
 def make_inputs(w: Workload, seed: int = 0, with_do: bool | None = None, nthreads=None,
-                S: int | None = None) -> dict:
-    """Q, K, V (and dO) for a workload as bf16 bit patterns, [B, S, H, D] row-major.
+                S: int | None = None, Skv: int | None = None) -> dict:
+    """Q, K, V (and dO) for a workload as bf16 bit patterns: Q (and dO) [B, S, H, D],
+    K and V [B, Skv, H, D] (Skv = S for self-attention), row-major.
 
-    ``S`` overrides the workload's token count (small parity cases)."""
+    ``S`` / ``Skv`` override the workload's query / key token counts (small parity cases)."""
     S = w.S if S is None else S
+    if Skv is None:
+        Skv = w.kv_len if w.cross else S
     shape = (w.B, S, w.H, w.D)
+    kv_shape = (w.B, Skv, w.H, w.D)
     out = {"q": make_tensor(shape, seed, STREAM_Q, nthreads),
-           "k": make_tensor(shape, seed, STREAM_K, nthreads),
-           "v": make_tensor(shape, seed, STREAM_V, nthreads)}
+           "k": make_tensor(kv_shape, seed, STREAM_K, nthreads),
+           "v": make_tensor(kv_shape, seed, STREAM_V, nthreads)}
     heads = peaky_heads(w.H, w.peaky_frac, seed)
     if heads:
         q = out["q"]
