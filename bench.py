@@ -126,10 +126,24 @@ def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
     t0 = time.perf_counter()
     oracle.attn_fwd(x["q"], x["k"], x["v"], rows=rows)
     dt = time.perf_counter() - t0
-    flop = 4.0 * w.B * w.H * len(rows) * w.S * w.D
+    flop = 4.0 * w.B * w.H * len(rows) * w.kv_len * w.D
     return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{len(rows)} query rows x {w.B * w.H} (batch, head) pairs of {w.name} "
-                      f"against all {w.S} keys, fp64 numpy/BLAS, {dt:.2f} s"}
+                      f"against all {w.kv_len} keys, fp64 numpy/BLAS, {dt:.2f} s"}
+
+
+def metric_of(w) -> str:
+    if w.cross:
+        return ("cross-attention TFLOP/s (fwd 4*B*H*S*Skv*D + bwd 2.5x fwd)" if w.backward
+                else "cross-attention TFLOP/s (4*B*H*S*Skv*D)")
+    return METRIC if not w.backward else "attention TFLOP/s (fwd 4*B*H*S^2*D + bwd 2.5x fwd)"
+
+
+def workload_config(w) -> dict:
+    c = {"workload": w.name, "B": w.B, "S": w.S, "H": w.H, "D": w.D}
+    if w.cross:
+        c["Skv"] = w.kv_len
+    return c
 
 
 def run_reference(args, w):
@@ -142,12 +156,11 @@ def run_reference(args, w):
         cpu_baseline(w, rows_per_step, x=x)
     vals = [cpu_baseline(w, rows_per_step, x=x) for _ in range(args.steps)]
     v = statistics.median(r["value"] for r in vals)
-    flop_step = 4.0 * w.B * w.H * rows_per_step * w.S * w.D
-    line = {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+    flop_step = 4.0 * w.B * w.H * rows_per_step * w.kv_len * w.D
+    line = {"metric": metric_of(w), "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": flop_step / (v * 1e12) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "B": w.B, "S": w.S, "H": w.H, "D": w.D,
-                       "sample_rows_per_head": rows_per_step},
+            "config": {**workload_config(w), "sample_rows_per_head": rows_per_step},
             "cpu_baseline": {**vals[0], "value": v},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -169,17 +182,27 @@ def whole_job_tflops(world: int, flop_per_rank_step: float, steps: int, slowest_
     return world * flop_per_rank_step * steps / (slowest_ms * 1e-3) / 1e12
 
 
+def bwd_splits(w, dev) -> bool:
+    """Whether the cross-attention backward spreads each key tile over several CTAs: it does
+    when the key tiles alone give fewer than 4 waves of CTAs on the device's SMs."""
+    import torch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return -(-w.kv_len // 128) * w.H * w.B < 4 * sms
+
+
 class Path:
     """The calls one bench step makes for a workload, with their buffers.
 
     fwd workloads: one wan_attn_fwd; the training workload: wan_attn_fwd then
-    wan_attn_bwd; the 8-bit workload: one wan_attn_fwd_q8 (quantise + attend).
+    wan_attn_bwd; the 8-bit workload: one wan_attn_fwd_q8 (quantise + attend);
+    the cross-attention workloads: wan_attn_cross_fwd (then wan_attn_cross_bwd).
     """
 
     def __init__(self, wa, w, dev, x):
         import torch
         self.wa, self.w = wa, w
         shape = (w.B, w.S, w.H, w.D)
+        kv_shape = (w.B, w.kv_len, w.H, w.D)
 
         def pinned(bits):
             return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -193,13 +216,17 @@ class Path:
         self.outs = [self.o, self.lse]
         self.ws = None
         if w.backward:
-            self.grads = [torch.empty(shape, **bf) for _ in range(3)]
-            self.ws = torch.empty(wa.bwd_workspace_size(w.B, w.S, w.H, w.D), dtype=torch.uint8, device=dev)
+            self.grads = [torch.empty(shape, **bf), torch.empty(kv_shape, **bf), torch.empty(kv_shape, **bf)]
+            ws_bytes = (wa.cross_bwd_workspace_size(w.B, w.S, w.kv_len, w.H, w.D) if w.cross
+                        else wa.bwd_workspace_size(w.B, w.S, w.H, w.D))
+            self.ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
             self.outs = self.outs + self.grads
             self.flop = 3.5 * w.fwd_flop                   # forward + 2.5x forward for the backward
             self.dominant_flop = 2.5 * w.fwd_flop
-            self.kernel = "wan::bwd::bwd_main_kernel (timed with its prep and dQ kernels: one wan_attn_bwd call)"
-            self.launches_per_step = 4
+            call = "wan_attn_cross_bwd" if w.cross else "wan_attn_bwd"
+            self.kernel = f"wan::bwd::bwd_main_kernel (timed with its prep and finalise kernels: one {call} call)"
+            # fwd + prep + main + dQ; a split key tile adds the dK and dV finalise kernels
+            self.launches_per_step = 4 + (2 if w.cross and bwd_splits(w, dev) else 0)
             self.peak_key, self.dtype = "bf16", "bf16"
         elif w.q8:
             self.ws = torch.empty(wa.fwd_q8_workspace_size(w.B, w.S, w.H, w.D), dtype=torch.uint8, device=dev)
@@ -211,7 +238,7 @@ class Path:
         else:
             self.flop = w.fwd_flop
             self.dominant_flop = w.fwd_flop
-            self.kernel = "wan::fwd::attn_fwd_kernel"
+            self.kernel = "wan::fwd::attn_fwd_kernel" + (" (wan_attn_cross_fwd)" if w.cross else "")
             self.launches_per_step = 1
             self.peak_key, self.dtype = "bf16", "bf16"
         self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
@@ -220,18 +247,20 @@ class Path:
 
     def step(self, dom_events=None):
         wa, (q, k, v) = self.wa, self.dev_in[:3]
+        fwd = wa.cross_fwd if self.w.cross else wa.fwd
         if self.w.backward:
-            wa.fwd(q, k, v, self.o, self.lse)
+            fwd(q, k, v, self.o, self.lse)
             if dom_events:
                 dom_events[0].record()
-            wa.bwd(q, k, v, self.o, self.dev_in[3], self.lse, *self.grads, workspace=self.ws)
+            bwd = wa.cross_bwd if self.w.cross else wa.bwd
+            bwd(q, k, v, self.o, self.dev_in[3], self.lse, *self.grads, workspace=self.ws)
         else:
             if dom_events:
                 dom_events[0].record()
             if self.w.q8:
                 wa.fwd_q8(q, k, v, self.o, self.lse, workspace=self.ws)
             else:
-                wa.fwd(q, k, v, self.o, self.lse)
+                fwd(q, k, v, self.o, self.lse)
         if dom_events:
             dom_events[1].record()
 
@@ -321,11 +350,11 @@ def run_ours(args, w):
             peak_src = f"{peaks['source']} bf16 dense (burst)"
         in_gb = sum(t.numel() * t.element_size() for t in path.dev_in) / 1e9
         line = {
-            "metric": METRIC if not w.backward else "attention TFLOP/s (fwd 4*B*H*S^2*D + bwd 2.5x fwd)",
+            "metric": metric_of(w),
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": path.dtype, "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "S": w.S, "H": w.H, "D": w.D,
+            "config": {**workload_config(w),
                        "flop_per_step": path.flop, "parallelism": f"replicas{world}",
                        "l2": "inputs (%.2f GB) exceed the 126 MB L2; no flush" % in_gb},
             "gpu_launches": args.steps * path.launches_per_step,

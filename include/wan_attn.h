@@ -95,6 +95,52 @@ WAN_ATTN_API int wan_attn_bwd(const void* q, const void* k, const void* v, const
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Cross-attention forward, bf16: the DiT block's attention from the video
+ * tokens to the text condition ("Wan 2.1 ..." paper-podcast summary, section
+ * "干预与形式化": c_txt is umT5's 512-token text embedding, and the DiT
+ * backbone injects umT5 by cross-attention).  Same definition as wan_attn_fwd
+ * with the key index running over the Skv key/value tokens:
+ *     O = softmax(Q K^T / sqrt(D)) V,  Q [Sq x D] per (b, h), K, V [Skv x D].
+ *   q       : in,  bf16 [B, Sq, H, D]
+ *   k, v    : in,  bf16 [B, Skv, H, D] (already projected to the attention heads)
+ *   o       : out, bf16 [B, Sq, H, D]
+ *   lse     : out, fp32 [B, H, Sq], natural log; not NULL
+ *   B, Sq, Skv, H >= 1 (each of B*Sq*H*D and B*Skv*H*D < 2^40); D must be 128.
+ * No mask: the Skv keys are all attended to (a caller whose text is padded
+ * passes the padded embedding, as the 512-token condition is).  Other
+ * conventions, precision and errors as wan_attn_fwd; wan_attn_cross_fwd with
+ * Skv = Sq and the same pointers computes what wan_attn_fwd does.
+ */
+WAN_ATTN_API int wan_attn_cross_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                    int Sq, int Skv, int H, int D, void* stream);
+
+/*
+ * Bytes of device workspace wan_attn_cross_bwd needs: fp32 dQ accumulator
+ * [B, Sq, H, D], fp32 D_i [B, H, Sq], fp32 dK and dV accumulators
+ * [B, Skv, H, D], each starting on a 256-byte boundary.  0 if the sizes are
+ * invalid.
+ */
+WAN_ATTN_API size_t wan_attn_cross_bwd_workspace_size(int B, int Sq, int Skv, int H, int D);
+
+/*
+ * Cross-attention backward, bf16: gradients of sum(O * dO) for
+ * O = wan_attn_cross_fwd(Q, K, V), with the formulas of wan_attn_bwd.
+ *   q, o, dO : in,  bf16 [B, Sq, H, D];  k, v : in, bf16 [B, Skv, H, D]
+ *   lse      : in,  fp32 [B, H, Sq] from wan_attn_cross_fwd on the same inputs
+ *   dq       : out, bf16 [B, Sq, H, D];  dk, dv : out, bf16 [B, Skv, H, D]
+ *   workspace, workspace_bytes : caller-owned device memory, 256-byte aligned,
+ *             at least wan_attn_cross_bwd_workspace_size bytes (else
+ *             WAN_ATTN_ERR_WORKSPACE); contents on entry ignored.
+ * With few key tiles (Skv = 512 gives 4 per head) the call spreads each key
+ * tile's queries over several CTAs that add their dK, dV parts in fp32 in the
+ * workspace; dK and dV (like dQ) may then differ in their low bits between
+ * runs.  Other conventions and errors as wan_attn_bwd.
+ */
+WAN_ATTN_API int wan_attn_cross_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                                    const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Skv,
+                                    int H, int D, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Bytes of device workspace wan_attn_fwd_q8 needs: the quantised copies and
  * their scales, each part starting on a 256-byte boundary, in this order:
  *   int8 Q8 [B, H, S, D], int8 K8 [B, H, S, D], e4m3 V8 [B, H, S, D],

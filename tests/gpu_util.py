@@ -33,3 +33,13 @@ def inputs_for(B, S, H, D=128, seed=0, with_do=False, q_mul=1.0):
     if with_do:
         x["do"] = synth.make_tensor(shape, seed, synth.STREAM_DO)
     return x
+
+
+def inputs_for_cross(B, Sq, Skv, H, D=128, seed=0, with_do=False):
+    """Q (and dO) [B, Sq, H, D], K and V [B, Skv, H, D] from the seeded generator."""
+    x = {"q": synth.make_tensor((B, Sq, H, D), seed, synth.STREAM_Q),
+         "k": synth.make_tensor((B, Skv, H, D), seed, synth.STREAM_K),
+         "v": synth.make_tensor((B, Skv, H, D), seed, synth.STREAM_V)}
+    if with_do:
+        x["do"] = synth.make_tensor((B, Sq, H, D), seed, synth.STREAM_DO)
+    return x

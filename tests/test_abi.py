@@ -103,3 +103,32 @@ def test_q8_host_side_validation_without_gpu(built):
     assert lib.wan_attn_fwd_q8(q, k, v, o, lse, 1, 130, 2, 128, ws, need - 1, None) == 5
     assert lib.wan_attn_fwd_q8(q, k, v, q, lse, 1, 130, 2, 128, ws, need, None) == 1
     assert lib.wan_attn_fwd_q8(q, k, v, o, lse, 1, 130, 2, 120, ws, need, None) == 2
+
+
+def test_cross_host_side_validation_without_gpu(built):
+    from video_dit_full_b200 import wan_attn
+    lib = wan_attn.lib()
+    INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 5
+    q, k, v, o, lse = (ctypes.c_void_p(0x100000 + i * 0x10000000) for i in range(5))
+    kv_bytes = 1 * 77 * 2 * 128 * 2
+    # Skv is validated on its own, and K, V are sized by it
+    assert lib.wan_attn_cross_fwd(q, k, v, o, lse, 1, 300, 0, 2, 128, None) == INVALID
+    assert lib.wan_attn_cross_fwd(q, k, v, o, lse, 1, 300, 77, 2, 64, None) == UNSUPPORTED
+    assert lib.wan_attn_cross_fwd(q, k, v, ctypes.c_void_p(k.value + kv_bytes - 256), lse, 1, 300, 77, 2, 128,
+                                  None) == INVALID     # o starts inside k
+    # workspace: dQ acc [Sq] + D_i [Sq] + dK, dV accumulators [Skv]
+    need = lib.wan_attn_cross_bwd_workspace_size(1, 300, 77, 2, 128)
+    a = lambda x: (x + 255) // 256 * 256
+    assert need == a(300 * 2 * 128 * 4) + a(2 * 300 * 4) + 2 * a(77 * 2 * 128 * 4)
+    assert lib.wan_attn_cross_bwd_workspace_size(1, 300, 0, 2, 128) == 0
+    ptr = [ctypes.c_void_p(0x100000 + i * 0x1000000) for i in range(10)]
+    q, k, v, o, do, lse, dq, dk, dv, ws = ptr
+    args = lambda **kw: [kw.get(n, d) for n, d in zip(
+        ["q", "k", "v", "o", "do", "lse", "dq", "dk", "dv", "B", "Sq", "Skv", "H", "D", "ws", "wsb", "st"],
+        [q, k, v, o, do, lse, dq, dk, dv, 1, 300, 77, 2, 128, ws, need, None])]
+    assert lib.wan_attn_cross_bwd(*args(ws=None)) == WORKSPACE
+    assert lib.wan_attn_cross_bwd(*args(wsb=need - 1)) == WORKSPACE
+    assert lib.wan_attn_cross_bwd(*args(Skv=-1)) == INVALID
+    assert lib.wan_attn_cross_bwd(*args(D=256)) == UNSUPPORTED
+    assert lib.wan_attn_cross_bwd(*args(dk=v)) == INVALID                 # output aliases an input
+    assert lib.wan_attn_cross_bwd(*args(dv=ctypes.c_void_p(dk.value + 64))) == INVALID   # outputs overlap

@@ -1,8 +1,8 @@
-"""B200 (sm_100a) full spatio-temporal self-attention for Wan-style video DiTs.
+"""B200 (sm_100a) full spatio-temporal self-attention (and the text cross-attention) for Wan-style video DiTs.
 
 The computation lives in ``libwan_attn.so`` (hand-written CUDA for sm_100a,
 C ABI in ``include/wan_attn.h``); ``wan_attn`` is its ctypes binding.
 """
-from .wan_attn import (WanAttnError, bwd, bwd_workspace_size, check_status, fwd, fwd_q8, fwd_q8_workspace_size, lib,
-                       q8_workspace_views, selftest_wait_timeout,  # noqa: F401
-                       set_wait_budget_ns, sync_status)
+from .wan_attn import (WanAttnError, bwd, bwd_workspace_size, check_status, cross_bwd,  # noqa: F401
+                       cross_bwd_workspace_size, cross_fwd, fwd, fwd_q8, fwd_q8_workspace_size, lib,
+                       q8_workspace_views, selftest_wait_timeout, set_wait_budget_ns, sync_status)

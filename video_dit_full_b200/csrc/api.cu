@@ -89,6 +89,20 @@ bool make_dq_acc_map(CUtensorMap* m, void* base, int B, int S, int H) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map over an fp32 [B, S, H, 128] accumulator as 4-D (128, H, S, B), box (32, 1, 128, 1)
+// with the 128-byte swizzle: the split backward adds [128 key][32 d] sub-tiles of dK, dV into it.
+bool make_acc_sw_map(CUtensorMap* m, void* base, int B, int S, int H) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {128 * 4, (cuuint64_t)H * 128 * 4, (cuuint64_t)S * H * 128 * 4};
+    const cuuint32_t box[4] = {32, 1, 128, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Range {
     uintptr_t lo, hi;
 };
@@ -149,31 +163,34 @@ __global__ void selftest_wait_kernel(unsigned long long budget_ns, int* status) 
 
 using namespace wan;
 
-extern "C" {
+namespace {
 
-int wan_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S, int H, int D,
-                 void* stream) {
+// Forward of Sq queries against Skv keys (self-attention: Skv = Sq).
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq, int Skv, int H,
+             int D, void* stream) {
     if (!q || !k || !v || !o || !lse) return WAN_ATTN_ERR_INVALID_ARG;
-    const int st = check_shape(B, S, H, D);
+    int st = check_shape(B, Sq, H, D);
+    if (st == WAN_ATTN_OK) st = check_shape(B, Skv, H, D);
     if (st != WAN_ATTN_OK) return st;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return WAN_ATTN_ERR_INVALID_ARG;
-    const size_t n = size_t(B) * S * H * D;
-    const Range rq = range_of(q, n * 2), rk = range_of(k, n * 2), rv = range_of(v, n * 2);
-    const Range ro = range_of(o, n * 2), rl = range_of(lse, size_t(B) * H * S * 4);
+    const size_t nq = size_t(B) * Sq * H * D, nkv = size_t(B) * Skv * H * D;
+    const Range rq = range_of(q, nq * 2), rk = range_of(k, nkv * 2), rv = range_of(v, nkv * 2);
+    const Range ro = range_of(o, nq * 2), rl = range_of(lse, size_t(B) * H * Sq * 4);
     for (const Range& in : {rq, rk, rv})
         if (overlaps(ro, in) || overlaps(rl, in)) return WAN_ATTN_ERR_INVALID_ARG;
     if (overlaps(ro, rl)) return WAN_ATTN_ERR_INVALID_ARG;
 
     CUtensorMap tq, tk, tv;
-    if (!make_bshd_map(&tq, q, B, S, H, D, 128) || !make_bshd_map(&tk, k, B, S, H, D, 128) ||
-        !make_bshd_map(&tv, v, B, S, H, D, 128))
+    if (!make_bshd_map(&tq, q, B, Sq, H, D, 128) || !make_bshd_map(&tk, k, B, Skv, H, D, 128) ||
+        !make_bshd_map(&tv, v, B, Skv, H, D, 128))
         return WAN_ATTN_ERR_CUDA;
     FwdParams p;
     p.o = o;
     p.lse = lse;
     p.B = B;
-    p.S = S;
+    p.S = Sq;
+    p.Skv = Skv;
     p.H = H;
     p.scale_log2 = static_cast<float>((1.0 / std::sqrt(double(D))) * 1.4426950408889634);
     p.wait_budget_ns = wait_budget_ns();
@@ -182,28 +199,33 @@ int wan_attn_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     return launch_fwd(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
 }
 
-size_t wan_attn_bwd_workspace_size(int B, int S, int H, int D) {
-    if (check_shape(B, S, H, D) != WAN_ATTN_OK) return 0;
-    const size_t n = size_t(B) * S * H * D;
-    return align256(n * 4) + align256(size_t(B) * H * S * 4);
+// Backward workspace: fp32 dQ accumulator [B, Sq, H, D], fp32 D_i [B, H, Sq] and, for the
+// cross-attention call, fp32 dK and dV accumulators [B, Skv, H, D]; each part 256-byte aligned.
+size_t bwd_ws_size(int B, int Sq, int Skv, int H, int D, bool cross) {
+    if (check_shape(B, Sq, H, D) != WAN_ATTN_OK || check_shape(B, Skv, H, D) != WAN_ATTN_OK) return 0;
+    const size_t nq = size_t(B) * Sq * H * D, nkv = size_t(B) * Skv * H * D;
+    size_t bytes = align256(nq * 4) + align256(size_t(B) * H * Sq * 4);
+    if (cross) bytes += 2 * align256(nkv * 4);
+    return bytes;
 }
 
-int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-                 void* dq, void* dk, void* dv, int B, int S, int H, int D, void* workspace,
-                 size_t workspace_bytes, void* stream) {
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+             void* dq, void* dk, void* dv, int B, int Sq, int Skv, int H, int D, void* workspace,
+             size_t workspace_bytes, void* stream, bool cross) {
     if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return WAN_ATTN_ERR_INVALID_ARG;
-    const int st = check_shape(B, S, H, D);
+    int st = check_shape(B, Sq, H, D);
+    if (st == WAN_ATTN_OK) st = check_shape(B, Skv, H, D);
     if (st != WAN_ATTN_OK) return st;
     for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(lse), static_cast<const void*>(dq),
                             static_cast<const void*>(dk), static_cast<const void*>(dv)})
         if (!aligned16(ptr)) return WAN_ATTN_ERR_INVALID_ARG;
-    const size_t need = wan_attn_bwd_workspace_size(B, S, H, D);
+    const size_t need = bwd_ws_size(B, Sq, Skv, H, D, cross);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return WAN_ATTN_ERR_WORKSPACE;
-    const size_t n = size_t(B) * S * H * D;
-    const Range ins[] = {range_of(q, n * 2), range_of(k, n * 2), range_of(v, n * 2), range_of(o, n * 2),
-                         range_of(dO, n * 2), range_of(lse, size_t(B) * H * S * 4)};
-    const Range outs[] = {range_of(dq, n * 2), range_of(dk, n * 2), range_of(dv, n * 2),
+    const size_t nq = size_t(B) * Sq * H * D, nkv = size_t(B) * Skv * H * D;
+    const Range ins[] = {range_of(q, nq * 2), range_of(k, nkv * 2), range_of(v, nkv * 2), range_of(o, nq * 2),
+                         range_of(dO, nq * 2), range_of(lse, size_t(B) * H * Sq * 4)};
+    const Range outs[] = {range_of(dq, nq * 2), range_of(dk, nkv * 2), range_of(dv, nkv * 2),
                           range_of(workspace, need)};
     for (size_t a = 0; a < 4; ++a) {
         for (const Range& in : ins)
@@ -212,27 +234,75 @@ int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, con
             if (overlaps(outs[a], outs[c])) return WAN_ATTN_ERR_INVALID_ARG;
     }
 
-    CUtensorMap tq, tk, tv, tdo, tdq;
-    if (!make_bshd_map(&tq, q, B, S, H, D, 128) || !make_bshd_map(&tk, k, B, S, H, D, 128) ||
-        !make_bshd_map(&tv, v, B, S, H, D, 128) || !make_bshd_map(&tdo, dO, B, S, H, D, 128) ||
-        !make_dq_acc_map(&tdq, workspace, B, S, H))
-        return WAN_ATTN_ERR_CUDA;
+    char* ws = static_cast<char*>(workspace);
+    const size_t off_delta = align256(nq * 4);
+    const size_t off_dk = off_delta + align256(size_t(B) * H * Sq * 4);
+    const size_t off_dv = off_dk + align256(nkv * 4);
     BwdParams p;
     p.lse = lse;
-    p.dq_acc = static_cast<float*>(workspace);
-    p.delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(n * 4));
+    p.dq_acc = reinterpret_cast<float*>(ws);
+    p.delta = reinterpret_cast<float*>(ws + off_delta);
+    p.dk_acc = cross ? reinterpret_cast<float*>(ws + off_dk) : nullptr;
+    p.dv_acc = cross ? reinterpret_cast<float*>(ws + off_dv) : nullptr;
+    CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
+    if (!make_bshd_map(&tq, q, B, Sq, H, D, 128) || !make_bshd_map(&tk, k, B, Skv, H, D, 128) ||
+        !make_bshd_map(&tv, v, B, Skv, H, D, 128) || !make_bshd_map(&tdo, dO, B, Sq, H, D, 128) ||
+        !make_dq_acc_map(&tdq, workspace, B, Sq, H))
+        return WAN_ATTN_ERR_CUDA;
+    if (cross) {
+        if (!make_acc_sw_map(&tdk, p.dk_acc, B, Skv, H) || !make_acc_sw_map(&tdv, p.dv_acc, B, Skv, H))
+            return WAN_ATTN_ERR_CUDA;
+    } else {
+        tdk = tdq;    // never read: self-attention keeps one CTA per key tile (nsplit = 1)
+        tdv = tdq;
+    }
     p.dk = dk;
     p.dv = dv;
     p.B = B;
-    p.S = S;
+    p.Sq = Sq;
+    p.Skv = Skv;
     p.H = H;
+    p.nsplit = 1;
     p.scale = static_cast<float>(1.0 / std::sqrt(double(D)));
     p.scale_log2 = static_cast<float>((1.0 / std::sqrt(double(D))) * 1.4426950408889634);
     p.wait_budget_ns = wait_budget_ns();
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
-    return launch_bwd(tq, tk, tv, tdo, tdq, p, o, dO, dq, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
-                                                                                          : WAN_ATTN_ERR_CUDA;
+    return launch_bwd(tq, tk, tv, tdo, tdq, tdk, tdv, p, cross, o, dO, dq, static_cast<cudaStream_t>(stream)) == 0
+               ? WAN_ATTN_OK
+               : WAN_ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int wan_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S, int H, int D,
+                 void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, S, S, H, D, stream);
+}
+
+int wan_attn_cross_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq, int Skv,
+                       int H, int D, void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, Sq, Skv, H, D, stream);
+}
+
+size_t wan_attn_bwd_workspace_size(int B, int S, int H, int D) { return bwd_ws_size(B, S, S, H, D, false); }
+
+int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int S, int H, int D, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, S, S, H, D, workspace, workspace_bytes, stream, false);
+}
+
+size_t wan_attn_cross_bwd_workspace_size(int B, int Sq, int Skv, int H, int D) {
+    return bwd_ws_size(B, Sq, Skv, H, D, true);
+}
+
+int wan_attn_cross_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                       const float* lse, void* dq, void* dk, void* dv, int B, int Sq, int Skv, int H, int D,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, Sq, Skv, H, D, workspace, workspace_bytes, stream, true);
 }
 
 size_t wan_attn_fwd_q8_workspace_size(int B, int S, int H, int D) {

@@ -20,6 +20,13 @@
 //                                       the accumulator (a dedicated reducer warp)
 //               P is recomputed from the forward's LSE; nothing of size S x S is stored.
 //   bwd_dq      dQ = bf16(accumulator / sqrt(D)).
+//
+// Queries and keys may differ in length (Sq, Skv): the block's cross-attention to the
+// 512-token umT5 text embedding ("Wan 2.1 ... paper-podcast summary", section
+// "干预与形式化").  With few key tiles (Skv = 512 gives 4 per head) one CTA per key tile
+// would leave most SMs idle, so the caller may split each key tile's Q range over nsplit
+// CTAs: each then adds its partial dK, dV into fp32 accumulators by TMA reduce-add (as dQ),
+// and bwd_dq converts those too.  With nsplit = 1 each CTA writes its dK, dV tiles in bf16.
 #include <cuda.h>
 
 #include "sm100_ptx.cuh"
@@ -44,7 +51,10 @@ constexpr int VEC_BYTES = 2 * 64 * 4;
 constexpr int OFF_BAR = OFF_VEC + 8 * VEC_BYTES;
 enum Bar { KV_FULL = 0, QDO_FULL = 1, QDO_EMPTY = 3, S_FULL = 5, DP_FULL = 6, P_READY = 7, DV_DONE = 8,
            DS_READY = 9, DQ_FULL = 10, DQ_DRAINED = 11, FINAL = 12, DRAIN = 13, STAGED = 14, DS_SMEM = 15,
-           NBARS = 16 };
+           RED_DONE = 16, EPI_STAGED = 17, NBARS = 18 };
+// split epilogue: dV (stage 0) and dK (stage 1) as four [128 key][32 d] fp32 sub-tiles each,
+// 128-byte swizzled, one TMA reduce-add per sub-tile
+constexpr int SUB_BYTES = BM * 32 * 4;
 constexpr int OFF_TMEM_SLOT = OFF_BAR + NBARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
 constexpr int SMEM_USED = OFF_ABORT + 8;
@@ -99,7 +109,8 @@ __device__ __forceinline__ void mma_ss_mn(uint32_t d_tmem, uint32_t a_smem, uint
 __global__ void __launch_bounds__(NTHREADS, 1)
 bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
-                const __grid_constant__ CUtensorMap tmdq, const BwdParams p) {
+                const __grid_constant__ CUtensorMap tmdq, const __grid_constant__ CUtensorMap tmdk,
+                const __grid_constant__ CUtensorMap tmdv, const BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -107,10 +118,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 
     const int warp = warp_id();
     const int lane = lane_id();
-    const int h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y;
+    const int b = blockIdx.z / p.nsplit, split = blockIdx.z % p.nsplit;
     const int kv0 = blockIdx.x * BM;
-    const int S = p.S;
-    const int nq = (S + BM - 1) / BM;
+    const int Sq = p.Sq, Skv = p.Skv;
+    // this CTA's Q tiles: [i_first, i_first + nq) of the (b, h)'s nq_all (nsplit <= nq_all)
+    const int nq_all = (Sq + BM - 1) / BM;
+    const int i_first = static_cast<int>(static_cast<long long>(split) * nq_all / p.nsplit);
+    const int nq = static_cast<int>(static_cast<long long>(split + 1) * nq_all / p.nsplit) - i_first;
 
     const uint32_t sK = base + OFF_K, sV = base + OFF_V;
     auto sQ = [&](int s) { return base + OFF_STAGE + s * STAGE_BYTES; };
@@ -137,6 +152,8 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         mbar_init(bar(FINAL), 1);
         mbar_init(bar(DRAIN), 1);
         mbar_init(bar(STAGED), G_THREADS);
+        mbar_init(bar(RED_DONE), 1);
+        mbar_init(bar(EPI_STAGED), G_THREADS);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -171,10 +188,11 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (!ok) break;
                 const uint32_t fb = bar(QDO_FULL + s);
                 mbar_arrive_expect_tx(fb, 2 * TILE_BYTES);
-                tma_load_4d_hint(sQ(s), &tmq, fb, 0, h, i * BM, b, keep);
-                tma_load_4d_hint(sQ(s) + HALF_BYTES, &tmq, fb, 64, h, i * BM, b, keep);
-                tma_load_4d_hint(sDO(s), &tmdo, fb, 0, h, i * BM, b, keep);
-                tma_load_4d_hint(sDO(s) + HALF_BYTES, &tmdo, fb, 64, h, i * BM, b, keep);
+                const int q_tok = (i_first + i) * BM;
+                tma_load_4d_hint(sQ(s), &tmq, fb, 0, h, q_tok, b, keep);
+                tma_load_4d_hint(sQ(s) + HALF_BYTES, &tmq, fb, 64, h, q_tok, b, keep);
+                tma_load_4d_hint(sDO(s), &tmdo, fb, 0, h, q_tok, b, keep);
+                tma_load_4d_hint(sDO(s) + HALF_BYTES, &tmdo, fb, 64, h, q_tok, b, keep);
                 par[s] = use;
             }
             if (!ok) {
@@ -227,12 +245,26 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             for (int i = 0; i < nq && ok; ++i) {
                 ok = wait_thread(bar(STAGED), i & 1, wc);
                 if (!ok) break;
-                tma_reduce_add_4d(&tmdq, base + OFF_STAGE + (i & 1) * STAGE_BYTES, 0, h, i * BM, b);
+                tma_reduce_add_4d(&tmdq, base + OFF_STAGE + (i & 1) * STAGE_BYTES, 0, h, (i_first + i) * BM, b);
                 bulk_commit_group();
                 bulk_wait_read_all();                         // the stage may be refilled now
                 mbar_arrive(bar(QDO_EMPTY + (i & 1)));
             }
             bulk_wait_all();
+            if (p.nsplit > 1 && ok) {
+                // split Q range: add this CTA's dV and dK tiles into the fp32 accumulators
+                mbar_arrive(bar(RED_DONE));                   // the stages are free for them
+                ok = wait_thread(bar(EPI_STAGED), 0, wc);
+                if (ok) {
+                    for (int which = 0; which < 2; ++which)
+                        for (int st = 0; st < 4; ++st)
+                            tma_reduce_add_4d(which ? &tmdk : &tmdv,
+                                              base + OFF_STAGE + which * STAGE_BYTES + st * SUB_BYTES, st * 32, h,
+                                              kv0, b);
+                    bulk_commit_group();
+                    bulk_wait_all();
+                }
+            }
         }
     } else {
         // -------- gradient warps: two threads per key row (or per d for dQ^T) -------
@@ -245,7 +277,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + T_S + lane_off + cb, tDP = tmem + T_DP + lane_off + cb;
         const int key = kv0 + j;
-        const bool key_ok = key < S;
+        const bool key_ok = key < Skv;
         const float c = p.scale_log2;
         const size_t bh = static_cast<size_t>(b) * p.H + h;
         // each warp keeps its own copy of its 64 queries' lse / D (no cross-warp barrier needed)
@@ -257,9 +289,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int col = e * 32 + lane;
-                const int qi = i * BM + cb + col;
-                s_lse[col] = qi < S ? p.lse[bh * S + qi] * LOG2E : INFINITY;
-                s_del[col] = qi < S ? p.delta[bh * S + qi] : 0.f;
+                const int qi = (i_first + i) * BM + cb + col;
+                s_lse[col] = qi < Sq ? p.lse[bh * Sq + qi] * LOG2E : INFINITY;
+                s_del[col] = qi < Sq ? p.delta[bh * Sq + qi] : 0.f;
             }
             __syncwarp();
 
@@ -343,9 +375,34 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             mbar_arrive(bar(STAGED));
         }
         if (ok) ok = wait_warp(bar(FINAL), 0, wc);
-        if (ok) {
+        if (ok && p.nsplit > 1) {
+            // stage dV, dK (fp32, unscaled) for the reducer warp's TMA reduce-adds, once it has
+            // finished reading the stages for dQ
+            ok = wait_warp(bar(RED_DONE), 0, wc);
+            if (ok) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int which = 0; which < 2; ++which) {
+                    const uint32_t src = tmem + (which ? T_DK : T_DV) + lane_off + cb;
+#pragma unroll 1
+                    for (int q = 0; q < 2; ++q) {
+                        uint32_t v[32];
+                        tmem_ld32(src + q * 32, v);
+                        tmem_wait_ld();
+                        // sub-tile hq*2+q holds d = 32(hq*2+q) .. +31; row j, 16-byte chunk c at c ^ (j % 8)
+                        uint8_t* row = smem + OFF_STAGE + which * STAGE_BYTES + (hq * 2 + q) * SUB_BYTES + j * 128;
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch)
+                            *reinterpret_cast<uint4*>(row + ((ch ^ (j & 7)) * 16)) =
+                                make_uint4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+                    }
+                }
+                fence_async_smem();
+                mbar_arrive(bar(EPI_STAGED));
+            }
+        } else if (ok) {
             tc_fence_after();
-            const size_t row = ((static_cast<size_t>(b) * S + key) * p.H + h) * HD + cb;
+            const size_t row = ((static_cast<size_t>(b) * Skv + key) * p.H + h) * HD + cb;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 const uint32_t src = tmem + (which ? T_DK : T_DV) + lane_off + cb;
@@ -443,23 +500,48 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ a
 }  // namespace bwd
 
 int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-               const CUtensorMap& tdq, const BwdParams& p, const void* o, const void* dout, void* dq,
-               cudaStream_t stream) {
-    const long long rows = static_cast<long long>(p.B) * p.S * p.H;
+               const CUtensorMap& tdq, const CUtensorMap& tdk, const CUtensorMap& tdv, BwdParams p,
+               bool allow_split, const void* o, const void* dout, void* dq, cudaStream_t stream) {
+    const long long rows = static_cast<long long>(p.B) * p.Sq * p.H;
+    const long long kv_rows = static_cast<long long>(p.B) * p.Skv * p.H;
     int sms = 148;
     int dev = 0;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // Split each key tile's Q range when the key tiles alone give fewer than 4 waves of CTAs:
+    // then aim at >= 8 waves (whole waves matter less as the count grows).
+    const int nkv = (p.Skv + bwd::BM - 1) / bwd::BM;
+    const int nq_all = (p.Sq + bwd::BM - 1) / bwd::BM;
+    const long long ctas = static_cast<long long>(nkv) * p.H * p.B;
+    int ns = 1;
+    if (allow_split && ctas < 4LL * sms) {
+        ns = static_cast<int>((8LL * sms + ctas - 1) / ctas);
+        if (ns > nq_all) ns = nq_all;
+        while (ns > 1 && static_cast<long long>(p.B) * ns > 65535) --ns;
+    }
+    p.nsplit = ns;
     const int ew_blocks = sms * 8;     // grid-stride elementwise kernels: 8 blocks of 256 per SM
     bwd::bwd_prep_kernel<<<ew_blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                         static_cast<const __nv_bfloat16*>(dout), p.delta, p.dq_acc,
-                                                        rows, p.S, p.H);
+                                                        rows, p.Sq, p.H);
     if (cudaGetLastError() != cudaSuccess) return -1;
+    if (ns > 1) {
+        const size_t acc_bytes = static_cast<size_t>(kv_rows) * bwd::HD * 4;
+        if (cudaMemsetAsync(p.dk_acc, 0, acc_bytes, stream) != cudaSuccess ||
+            cudaMemsetAsync(p.dv_acc, 0, acc_bytes, stream) != cudaSuccess)
+            return -1;
+    }
     if (configure_smem(reinterpret_cast<const void*>(bwd::bwd_main_kernel), bwd::SMEM_BYTES) != 0) return -1;
-    const dim3 grid((p.S + bwd::BM - 1) / bwd::BM, p.H, p.B);
-    bwd::bwd_main_kernel<<<grid, bwd::NTHREADS, bwd::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
+    const dim3 grid(nkv, p.H, p.B * ns);
+    bwd::bwd_main_kernel<<<grid, bwd::NTHREADS, bwd::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
     if (cudaGetLastError() != cudaSuccess) return -1;
     bwd::bwd_dq_kernel<<<ew_blocks, 256, 0, stream>>>(p.dq_acc, static_cast<__nv_bfloat16*>(dq), rows * 16,
                                                       p.scale);
+    if (ns > 1) {
+        bwd::bwd_dq_kernel<<<ew_blocks, 256, 0, stream>>>(p.dk_acc, static_cast<__nv_bfloat16*>(p.dk), kv_rows * 16,
+                                                          p.scale);
+        bwd::bwd_dq_kernel<<<ew_blocks, 256, 0, stream>>>(p.dv_acc, static_cast<__nv_bfloat16*>(p.dv), kv_rows * 16,
+                                                          1.0f);
+    }
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

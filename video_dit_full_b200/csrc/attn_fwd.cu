@@ -4,7 +4,10 @@
 // What is computed: the DiT block's full spatio-temporal self-attention
 // ("Wan 2.1 ... paper-podcast summary", section "干预与形式化": full
 // spatio-temporal self-attention, neither windowed nor U-ViT; section
-// "先看现象": non-causal attention, forward cost term 4*b*s^2*h).
+// "先看现象": non-causal attention, forward cost term 4*b*s^2*h).  The same kernel
+// serves the block's cross-attention from the video tokens to the 512-token umT5
+// text embedding (same summary, section "干预与形式化"): queries and keys then
+// have different lengths (S and Skv).
 //
 // How (one CTA = two 128-row Q tiles of one (batch, head)):
 //   warp 8      TMA producer: Q tiles once, then K_j / V_j 128-key tiles into a
@@ -81,7 +84,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     const int h = blockIdx.y, b = blockIdx.z;
     const int q0 = blockIdx.x * (NQ * BM);
     const int nq = (q0 + BM < p.S) ? 2 : 1;          // second tile empty on a short tail
-    const int nkv = (p.S + BN - 1) / BN;
+    const int nkv = (p.Skv + BN - 1) / BN;
 
     const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sV = base + OFF_V;
     const uint32_t bar0 = base + OFF_BAR;
@@ -216,7 +219,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q * 32]));
             tmem_wait_ld();
             float* s = reinterpret_cast<float*>(sr);
-            const int valid = p.S - j * BN;      // keys of this tile that exist
+            const int valid = p.Skv - j * BN;    // keys of this tile that exist
             if (valid < BN) {
 #pragma unroll
                 for (int q = 0; q < 128; ++q)

@@ -151,7 +151,6 @@ constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
 constexpr int NTHREADS = 320;               // warps 0-3 softmax of Q tile 0, 4-7 of Q tile 1, 8 TMA, 9 MMA
 constexpr uint32_t TMEM_COLS = 512;         // S0 | S1 (int32; P8 over their first 32 columns) | O0 | O1
 constexpr uint32_t T_O = 256;
-constexpr float LOG2_448 = 8.807354922057604f;
 // The running max is moved only when it rises by more than 1 (log2 units), so p <= 2 against
 // the max in use; P is then quantised as e4m3(P_SCALE * p * sV_block / sV_max) <= 448.
 constexpr float RESCALE_THRESHOLD = 1.0f;

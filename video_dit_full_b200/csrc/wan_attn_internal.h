@@ -12,19 +12,23 @@ namespace wan {
 struct FwdParams {
     void* o;                    // bf16 [B, S, H, 128]
     float* lse;                 // fp32 [B, H, S], natural log
-    int B, S, H;
+    int B, S, H;                // S = query tokens
+    int Skv;                    // key / value tokens (= S for self-attention)
     float scale_log2;           // (1 / sqrt(D)) * log2(e)
     unsigned long long wait_budget_ns;
     int* status;                // device status word (see wan_attn_sync_status)
 };
 
 struct BwdParams {
-    const float* lse;           // fp32 [B, H, S] from the forward (natural log)
-    float* delta;               // workspace fp32 [B, H, S]: rowsum(dO * O)
-    float* dq_acc;              // workspace fp32 [B, S, H, 128]: unscaled dS K
-    void* dk;                   // bf16 [B, S, H, 128]
-    void* dv;                   // bf16 [B, S, H, 128]
-    int B, S, H;
+    const float* lse;           // fp32 [B, H, Sq] from the forward (natural log)
+    float* delta;               // workspace fp32 [B, H, Sq]: rowsum(dO * O)
+    float* dq_acc;              // workspace fp32 [B, Sq, H, 128]: unscaled dS K
+    float* dk_acc;              // workspace fp32 [B, Skv, H, 128] (split query ranges only)
+    float* dv_acc;              // workspace fp32 [B, Skv, H, 128] (split query ranges only)
+    void* dk;                   // bf16 [B, Skv, H, 128]
+    void* dv;                   // bf16 [B, Skv, H, 128]
+    int B, Sq, Skv, H;
+    int nsplit;                 // CTAs sharing one key tile, each over its own range of Q tiles
     float scale;                // 1 / sqrt(D)
     float scale_log2;           // scale * log2(e)
     unsigned long long wait_budget_ns;
@@ -59,9 +63,12 @@ int configure_smem(const void* kernel, int bytes);
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                cudaStream_t stream);
 
+// Chooses p.nsplit (1 unless allow_split and the key tiles alone fill too few waves of the
+// GPU), then launches the backward's kernels.  tdk / tdv (fp32 accumulators, as tdq) are only
+// read when p.nsplit > 1.
 int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-               const CUtensorMap& tdq, const BwdParams& p, const void* o, const void* dout, void* dq,
-               cudaStream_t stream);
+               const CUtensorMap& tdq, const CUtensorMap& tdk, const CUtensorMap& tdv, BwdParams p,
+               bool allow_split, const void* o, const void* dout, void* dq, cudaStream_t stream);
 
 int launch_q8(const Q8QuantParams& qp, const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv8,
               const Q8AttnParams& p, cudaStream_t stream);

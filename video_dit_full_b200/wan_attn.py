@@ -23,6 +23,9 @@ SIGNATURES = [
     ("wan_attn_fwd", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P]),
     ("wan_attn_bwd_workspace_size", _Z, [_I, _I, _I, _I]),
     ("wan_attn_bwd", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]),
+    ("wan_attn_cross_fwd", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _P]),
+    ("wan_attn_cross_bwd_workspace_size", _Z, [_I, _I, _I, _I, _I]),
+    ("wan_attn_cross_bwd", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
     ("wan_attn_fwd_q8_workspace_size", _Z, [_I, _I, _I, _I]),
     ("wan_attn_fwd_q8", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P, _Z, _P]),
     ("wan_attn_bwd_noalloc", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _P]),
@@ -126,6 +129,64 @@ def bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None, stream=N
                                               do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
                                               dv.data_ptr(), B, S, H, D, workspace.data_ptr(),
                                               workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
+    return dq, dk, dv
+
+
+def _check_kv(q, k, v):
+    """K and V of a cross-attention call: [B, Skv, H, D] with q's B, H, D."""
+    _check_bshd("k", k)
+    B, _, H, D = q.shape
+    Skv = k.shape[1]
+    if (k.shape[0], k.shape[2], k.shape[3]) != (B, H, D):
+        raise ValueError(f"k has shape {tuple(k.shape)}, expected [B={B}, Skv, H={H}, D={D}]")
+    _check_bshd("v", v, k.shape)
+    return Skv
+
+
+def cross_fwd(q, k, v, o=None, lse=None, stream=None):
+    """O, LSE of q [B, Sq, H, D] attending to k, v [B, Skv, H, D] through ``wan_attn_cross_fwd``."""
+    import torch
+    _check_bshd("q", q)
+    B, Sq, H, D = q.shape
+    Skv = _check_kv(q, k, v)
+    o = torch.empty_like(q) if o is None else o
+    _check_bshd("o", o, q.shape)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Sq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, Sq] tensor")
+    _check("wan_attn_cross_fwd", lib().wan_attn_cross_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                                          lse.data_ptr(), B, Sq, Skv, H, D, _stream_ptr(stream)))
+    return o, lse
+
+
+def cross_bwd_workspace_size(B, Sq, Skv, H, D=128) -> int:
+    return lib().wan_attn_cross_bwd_workspace_size(B, Sq, Skv, H, D)
+
+
+def cross_bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of sum(O * dO) for the cross-attention through ``wan_attn_cross_bwd``."""
+    import torch
+    _check_bshd("q", q)
+    B, Sq, H, D = q.shape
+    Skv = _check_kv(q, k, v)
+    for name, t in (("o", o), ("do", do)):
+        _check_bshd(name, t, q.shape)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Sq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, Sq] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_bshd("dq", dq, q.shape)
+    _check_bshd("dk", dk, k.shape)
+    _check_bshd("dv", dv, k.shape)
+    if workspace is None:
+        workspace = torch.empty(cross_bwd_workspace_size(B, Sq, Skv, H, D), dtype=torch.uint8, device=q.device)
+    _check("wan_attn_cross_bwd",
+           lib().wan_attn_cross_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Sq, Skv, H, D,
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    _stream_ptr(stream)))
     return dq, dk, dv
 
 
