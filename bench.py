@@ -133,6 +133,8 @@ def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
 
 
 def metric_of(w) -> str:
+    if w.cp:
+        return f"{w.cp} context-parallel attention TFLOP/s per rank (4*B*H*S^2*D / {w.cp_ranks})"
     if w.cross:
         return ("cross-attention TFLOP/s (fwd 4*B*H*S*Skv*D + bwd 2.5x fwd)" if w.backward
                 else "cross-attention TFLOP/s (4*B*H*S*Skv*D)")
@@ -143,6 +145,8 @@ def workload_config(w) -> dict:
     c = {"workload": w.name, "B": w.B, "S": w.S, "H": w.H, "D": w.D}
     if w.cross:
         c["Skv"] = w.kv_len
+    if w.cp:
+        c.update(cp=w.cp, cp_ranks=w.cp_ranks, cp_note="one rank's kernels; the exchanges are not run")
     return c
 
 
@@ -272,6 +276,93 @@ class Path:
             h.copy_(d, non_blocking=True)
 
 
+class CpPath:
+    """One rank's compute of a G-way context split (Ring or Ulysses) on this GPU.
+
+    The other ranks' shards are already resident, so the exchanges (NCCL on a real
+    split) are not part of the step: it is the per-rank kernel work only.
+    ring:    G x (wan_attn_cross_fwd of the rank's S/G queries against one key block
+             + wan_attn_cp_merge into the fp32 running result).
+    ulysses: wan_attn_cp_layout of the q, k, v shards into send order, wan_attn_fwd on
+             all S tokens of the rank's H/G heads, wan_attn_cp_layout of O back into
+             sequence order (B = 1: the head-side permutations are identities).
+    """
+
+    def __init__(self, wa, w, dev, x):
+        import torch
+        self.wa, self.w = wa, w
+        G, B, S, H, D = w.cp_ranks, w.B, w.S, w.H, w.D
+        if B != 1 or S % G or H % G:
+            raise ValueError("context-parallel workloads need B = 1, S and H divisible by the ranks")
+        self.G, self.S_loc, self.Hg = G, S // G, H // G
+
+        def dev_bf16(bits):
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+        full = [dev_bf16(x[n]) for n in ("q", "k", "v")]
+        sl = slice(0, self.S_loc)
+        # this rank's own shards (its tokens 0..S/G-1 with every head): what e2e copies in
+        self.host_in = [torch.from_numpy(np.ascontiguousarray(x[n][:, sl]).view(np.int16)).view(torch.bfloat16)
+                        .pin_memory() for n in ("q", "k", "v")]
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        if w.cp == "ring":
+            self.dev_in = [t[:, sl] for t in full]           # views of the resident tensors (B = 1)
+            self.blocks = [(full[1][:, j * self.S_loc:(j + 1) * self.S_loc],
+                            full[2][:, j * self.S_loc:(j + 1) * self.S_loc]) for j in range(G)]
+            self.o = torch.empty((B, self.S_loc, H, D), **bf)
+            self.o_acc = torch.empty(self.o.shape, dtype=torch.float32, device=dev)
+            self.lse = torch.empty((B, H, self.S_loc), dtype=torch.float32, device=dev)
+            self.outs = [self.o, self.lse]
+            self.kernel = ("wan::fwd::attn_fwd_kernel + wan::cp::cp_merge_kernel (one rank's 8 key blocks: "
+                           "wan_attn_cross_fwd + wan_attn_cp_merge each)")
+            self.launches_per_step = 2 * G
+        else:
+            self.dev_in = [t[:, sl].contiguous() for t in full]   # own shards, [B, S/G, H, D]
+            # all tokens of this rank's head group, as the all-to-all would deliver them
+            self.heads = [t[:, :, :self.Hg].contiguous() for t in full]
+            self.send = [torch.empty((G, B, self.S_loc, self.Hg, D), **bf) for _ in range(3)]
+            self.o_heads = torch.empty((B, S, self.Hg, D), **bf)
+            self.lse_h = torch.empty((B, self.Hg, S), dtype=torch.float32, device=dev)
+            self.o = torch.empty((B, self.S_loc, H, D), **bf)
+            self.outs = [self.o]
+            self.kernel = ("wan::fwd::attn_fwd_kernel + wan::cp::cp_layout_kernel (one rank: 3 layouts in, "
+                           "attention on its 5 heads x all tokens, 1 layout out)")
+            self.launches_per_step = 5
+        del full
+        self.flop = w.fwd_flop
+        self.dominant_flop = w.fwd_flop
+        self.peak_key, self.dtype = "bf16", "bf16"
+        self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.host_in)
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.host_out)
+
+    def step(self, dom_events=None):
+        wa = self.wa
+        if dom_events:
+            dom_events[0].record()
+        if self.w.cp == "ring":
+            q = self.dev_in[0]
+            for j, (k, v) in enumerate(self.blocks):
+                o_t, lse_t = wa.cross_fwd(q, k, v)
+                wa.cp_merge(self.o_acc, self.lse, o_t, lse_t, j == 0, self.o if j + 1 == self.G else None)
+        else:
+            G, B, S_loc, Hg = self.G, self.w.B, self.S_loc, self.Hg
+            for send, shard in zip(self.send, self.dev_in):
+                wa.cp_layout(send, shard, B, S_loc, G, Hg, wa.CP_SEQ_TO_SEND)
+            wa.fwd(*self.heads, self.o_heads, self.lse_h)
+            # o_heads in [B, G*S_loc, Hg, D] is already the send order for B = 1
+            wa.cp_layout(self.o, self.o_heads, B, S_loc, G, Hg, wa.CP_RECV_TO_SEQ)
+        if dom_events:
+            dom_events[1].record()
+
+    def e2e_step(self):
+        for d, h in zip(self.dev_in, self.host_in):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        for h, d in zip(self.host_out, self.outs):
+            h.copy_(d, non_blocking=True)
+
+
 def run_ours(args, w):
     import torch
     import video_dit_full_b200 as wa
@@ -291,7 +382,7 @@ def run_ours(args, w):
 
     # each rank gets its own seeded problem (seed = rank): weak scaling
     x = synth.make_inputs(w, seed=rank)
-    path = Path(wa, w, dev, x)
+    path = CpPath(wa, w, dev, x) if w.cp else Path(wa, w, dev, x)
     stream = torch.cuda.current_stream(dev)
 
     def barrier():

@@ -141,6 +141,60 @@ WAN_ATTN_API int wan_attn_cross_bwd(const void* q, const void* k, const void* v,
                                     int H, int D, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Context parallelism: the building blocks of the two schemes the pages name for
+ * sequences too long for one GPU (kwkr.cn Wan explainer, section 3.2: the token
+ * sequence is split over GPUs and combined with Ulysses and Ring Attention;
+ * "Wan: Open and Advanced Large-Scale Video Generative Models", section 5: the
+ * DiT trains with FSDP + 2-D context parallel, converting layouts at module
+ * boundaries).  The exchanges themselves (all-to-all, ring send/recv) are NCCL
+ * calls made by the caller (video_dit_full_b200.context_parallel).
+ *
+ * Ring Attention.  A rank holding queries Q_r meets the key blocks K_t, V_t one
+ * at a time; wan_attn_cross_fwd gives each block's partial (O_t, lse_t) and
+ *     lse' = logaddexp(lse, lse_t),   O' = e^(lse - lse') O + e^(lse_t - lse') O_t
+ * folds it into a running fp32 (O, lse): exactly the softmax over every key
+ * seen so far.
+ *   o_acc    : in/out fp32 [B, S, H, D]   (ignored on input when first != 0)
+ *   lse_acc  : in/out fp32 [B, H, S]      (ignored on input when first != 0)
+ *   o_part   : in  bf16 [B, S, H, D];  lse_part : in fp32 [B, H, S] (natural log)
+ *   o_out    : out bf16 [B, S, H, D] = the updated o_acc rounded to nearest even,
+ *              or NULL for none
+ *   first    : non-zero = start a new sum (o_acc = o_part, lse_acc = lse_part)
+ *   D must be 128.  Pointers 16-byte aligned; outputs overlap nothing.
+ */
+WAN_ATTN_API int wan_attn_cp_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                                   void* o_out, int B, int S, int H, int D, int first, void* stream);
+
+/*
+ * acc = (first ? 0 : acc) + part over n elements (part bf16, acc fp32), and
+ * out = bf16(acc) when out is not NULL: the ring backward's sums of dQ parts
+ * and of the dK, dV parts that travel with their key block.  n must be a
+ * positive multiple of 8; pointers 16-byte aligned; no overlaps.
+ */
+WAN_ATTN_API int wan_attn_cp_accumulate(float* acc, const void* part, void* out, size_t n, int first,
+                                        void* stream);
+
+/*
+ * Ulysses.  A rank holds S_loc tokens of all H = G*Hg heads; one all-to-all
+ * (equal chunks, chunk g to rank g) gives every rank all G*S_loc tokens of its
+ * Hg heads, attention runs locally, and a second all-to-all brings O back.
+ * wan_attn_cp_layout moves [Hg x D] bf16 blocks between the orders around
+ * those exchanges (B = batch, g = rank / head group, s = token within a shard):
+ *   WAN_ATTN_CP_SEQ_TO_SEND   [B, S_loc, G, Hg, D] -> [G, B, S_loc, Hg, D]  (send buffer)
+ *   WAN_ATTN_CP_RECV_TO_HEADS [G, B, S_loc, Hg, D] -> [B, G*S_loc, Hg, D]   (attention input)
+ *   WAN_ATTN_CP_HEADS_TO_SEND [B, G*S_loc, Hg, D] -> [G, B, S_loc, Hg, D]   (send buffer)
+ *   WAN_ATTN_CP_RECV_TO_SEQ   [G, B, S_loc, Hg, D] -> [B, S_loc, G*Hg, D]   (back in sequence shards)
+ * dst and src hold B*S_loc*G*Hg*D bf16 each, 16-byte aligned, not overlapping;
+ * D must be 128.
+ */
+#define WAN_ATTN_CP_SEQ_TO_SEND 0
+#define WAN_ATTN_CP_RECV_TO_HEADS 1
+#define WAN_ATTN_CP_HEADS_TO_SEND 2
+#define WAN_ATTN_CP_RECV_TO_SEQ 3
+WAN_ATTN_API int wan_attn_cp_layout(void* dst, const void* src, int B, int S_loc, int G, int Hg, int D, int which,
+                                    void* stream);
+
+/*
  * Bytes of device workspace wan_attn_fwd_q8 needs: the quantised copies and
  * their scales, each part starting on a 256-byte boundary, in this order:
  *   int8 Q8 [B, H, S, D], int8 K8 [B, H, S, D], e4m3 V8 [B, H, S, D],

@@ -163,6 +163,8 @@ class Workload:
     backward: bool = False
     q8: bool = False
     Skv: int | None = None         # key/value tokens when they differ from S (cross-attention)
+    cp: str | None = None          # "ring" / "ulysses": one rank's share of a G-way context split
+    cp_ranks: int = 1
 
     @property
     def kv_len(self) -> int:
@@ -174,8 +176,9 @@ class Workload:
 
     @property
     def fwd_flop(self) -> float:
-        """4*B*H*S*Skv*D: the forward's two S x Skv x D contractions (multiply-add = 2)."""
-        return 4.0 * self.B * self.H * self.S * self.kv_len * self.D
+        """4*B*H*S*Skv*D: the forward's two S x Skv x D contractions (multiply-add = 2);
+        for a context-parallel workload, one rank's 1/G share of it."""
+        return 4.0 * self.B * self.H * self.S * self.kv_len * self.D / self.cp_ranks
 
 
 WORKLOADS = {
@@ -195,6 +198,11 @@ WORKLOADS = {
                            video=(81, 720, 1280), Skv=TEXT_TOKENS),
     "cross_train_480p": Workload("cross_train_480p", 1, tokens_for_video(81, 480, 832), 40, 128,
                                  video=(81, 480, 832), backward=True, Skv=TEXT_TOKENS),
+    # one rank's compute of the 720p attention split 8 ways (kwkr.cn Wan explainer, section 3.2)
+    "ring8_720p_rank": Workload("ring8_720p_rank", 1, tokens_for_video(81, 720, 1280), 40, 128,
+                                video=(81, 720, 1280), cp="ring", cp_ranks=8),
+    "ulysses8_720p_rank": Workload("ulysses8_720p_rank", 1, tokens_for_video(81, 720, 1280), 40, 128,
+                                   video=(81, 720, 1280), cp="ulysses", cp_ranks=8),
 }
 
 

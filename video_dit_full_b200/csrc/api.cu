@@ -369,6 +369,62 @@ int wan_attn_fwd_q8(const void* q, const void* k, const void* v, void* o, float*
     return launch_q8(qp, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
 }
 
+int wan_attn_cp_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                      int S, int H, int D, int first, void* stream) {
+    if (!o_acc || !lse_acc || !o_part || !lse_part) return WAN_ATTN_ERR_INVALID_ARG;
+    const int st = check_shape(B, S, H, D);
+    if (st != WAN_ATTN_OK) return st;
+    for (const void* ptr : {static_cast<const void*>(o_acc), static_cast<const void*>(lse_acc), o_part,
+                            static_cast<const void*>(lse_part), static_cast<const void*>(o_out)})
+        if (ptr && !aligned16(ptr)) return WAN_ATTN_ERR_INVALID_ARG;
+    const size_t n = size_t(B) * S * H * D, nl = size_t(B) * H * S;
+    const Range ra = range_of(o_acc, n * 4), rl = range_of(lse_acc, nl * 4);
+    const Range ins[] = {range_of(o_part, n * 2), range_of(lse_part, nl * 4)};
+    for (const Range& in : ins)
+        if (overlaps(ra, in) || overlaps(rl, in)) return WAN_ATTN_ERR_INVALID_ARG;
+    if (overlaps(ra, rl)) return WAN_ATTN_ERR_INVALID_ARG;
+    if (o_out) {
+        const Range ro = range_of(o_out, n * 2);
+        if (overlaps(ro, ra) || overlaps(ro, rl) || overlaps(ro, ins[0]) || overlaps(ro, ins[1]))
+            return WAN_ATTN_ERR_INVALID_ARG;
+    }
+    return launch_cp_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, S, H, first ? 1 : 0,
+                           static_cast<cudaStream_t>(stream)) == 0
+               ? WAN_ATTN_OK
+               : WAN_ATTN_ERR_CUDA;
+}
+
+int wan_attn_cp_accumulate(float* acc, const void* part, void* out, size_t n, int first, void* stream) {
+    if (!acc || !part || n == 0 || (n & 7u)) return WAN_ATTN_ERR_INVALID_ARG;
+    if (!aligned16(acc) || !aligned16(part) || (out && !aligned16(out))) return WAN_ATTN_ERR_INVALID_ARG;
+    const Range ra = range_of(acc, n * 4), rp = range_of(part, n * 2);
+    if (overlaps(ra, rp)) return WAN_ATTN_ERR_INVALID_ARG;
+    if (out) {
+        const Range ro = range_of(out, n * 2);
+        if (overlaps(ro, ra) || overlaps(ro, rp)) return WAN_ATTN_ERR_INVALID_ARG;
+    }
+    return launch_cp_accumulate(acc, part, out, static_cast<long long>(n / 8), first ? 1 : 0,
+                                static_cast<cudaStream_t>(stream)) == 0
+               ? WAN_ATTN_OK
+               : WAN_ATTN_ERR_CUDA;
+}
+
+int wan_attn_cp_layout(void* dst, const void* src, int B, int S_loc, int G, int Hg, int D, int which,
+                       void* stream) {
+    if (!dst || !src || G < 1 || Hg < 1 || which < WAN_ATTN_CP_SEQ_TO_SEND || which > WAN_ATTN_CP_RECV_TO_SEQ)
+        return WAN_ATTN_ERR_INVALID_ARG;
+    if (static_cast<long long>(G) * Hg > 65535) return WAN_ATTN_ERR_INVALID_ARG;
+    const int st = check_shape(B, S_loc, G * Hg, D);
+    if (st != WAN_ATTN_OK) return st;
+    if (double(B) * S_loc * G * Hg * D >= double(1ull << 40) / G) return WAN_ATTN_ERR_INVALID_ARG;
+    if (!aligned16(dst) || !aligned16(src)) return WAN_ATTN_ERR_INVALID_ARG;
+    const size_t bytes = size_t(B) * S_loc * G * Hg * D * 2;
+    if (overlaps(range_of(dst, bytes), range_of(src, bytes))) return WAN_ATTN_ERR_INVALID_ARG;
+    return launch_cp_layout(dst, src, B, S_loc, G, Hg * D * 2 / 16, which, static_cast<cudaStream_t>(stream)) == 0
+               ? WAN_ATTN_OK
+               : WAN_ATTN_ERR_CUDA;
+}
+
 int wan_attn_sync_status(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WAN_ATTN_ERR_CUDA;
     int h = 0;

@@ -70,6 +70,12 @@ int launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
                const CUtensorMap& tdq, const CUtensorMap& tdk, const CUtensorMap& tdv, BwdParams p,
                bool allow_split, const void* o, const void* dout, void* dq, cudaStream_t stream);
 
+// Context-parallel helpers (cp_kernels.cu).  0 on success.
+int launch_cp_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                    int S, int H, int first, cudaStream_t stream);
+int launch_cp_accumulate(float* acc, const void* part, void* out, long long n8, int first, cudaStream_t stream);
+int launch_cp_layout(void* dst, const void* src, int B, int S, int G, int blk16, int which, cudaStream_t stream);
+
 int launch_q8(const Q8QuantParams& qp, const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv8,
               const Q8AttnParams& p, cudaStream_t stream);
 

@@ -26,6 +26,9 @@ SIGNATURES = [
     ("wan_attn_cross_fwd", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _I, _P]),
     ("wan_attn_cross_bwd_workspace_size", _Z, [_I, _I, _I, _I, _I]),
     ("wan_attn_cross_bwd", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    ("wan_attn_cp_merge", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    ("wan_attn_cp_accumulate", _I, [_P, _P, _P, _Z, _I, _P]),
+    ("wan_attn_cp_layout", _I, [_P, _P, _I, _I, _I, _I, _I, _I, _P]),
     ("wan_attn_fwd_q8_workspace_size", _Z, [_I, _I, _I, _I]),
     ("wan_attn_fwd_q8", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P, _Z, _P]),
     ("wan_attn_bwd_noalloc", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _P]),
@@ -188,6 +191,57 @@ def cross_bwd(q, k, v, o, do, lse, dq=None, dk=None, dv=None, workspace=None, st
                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream_ptr(stream)))
     return dq, dk, dv
+
+
+CP_SEQ_TO_SEND, CP_RECV_TO_HEADS, CP_HEADS_TO_SEND, CP_RECV_TO_SEQ = 0, 1, 2, 3
+
+
+def _check_plain(name, t, dtype, numel=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {numel}")
+
+
+def cp_merge(o_acc, lse_acc, o_part, lse_part, first, o_out=None, stream=None):
+    """Fold a partial (o_part bf16 [B, S, H, D], lse_part fp32 [B, H, S]) into the fp32 running
+    (o_acc, lse_acc) through ``wan_attn_cp_merge``; o_out (bf16) receives the result if given."""
+    import torch
+    _check_bshd("o_part", o_part)
+    B, S, H, D = o_part.shape
+    _check_plain("o_acc", o_acc, torch.float32, o_part.numel())
+    _check_plain("lse_acc", lse_acc, torch.float32, B * H * S)
+    _check_plain("lse_part", lse_part, torch.float32, B * H * S)
+    if o_out is not None:
+        _check_bshd("o_out", o_out, o_part.shape)
+    _check("wan_attn_cp_merge", lib().wan_attn_cp_merge(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(),
+                                                        lse_part.data_ptr(), o_out.data_ptr() if o_out is not None
+                                                        else None, B, S, H, D, 1 if first else 0,
+                                                        _stream_ptr(stream)))
+
+
+def cp_accumulate(acc, part, first, out=None, stream=None):
+    """acc (fp32) = (0 if first else acc) + part (bf16); out = bf16(acc) if given."""
+    import torch
+    _check_plain("part", part, torch.bfloat16)
+    _check_plain("acc", acc, torch.float32, part.numel())
+    if out is not None:
+        _check_plain("out", out, torch.bfloat16, part.numel())
+    _check("wan_attn_cp_accumulate", lib().wan_attn_cp_accumulate(acc.data_ptr(), part.data_ptr(),
+                                                                  out.data_ptr() if out is not None else None,
+                                                                  part.numel(), 1 if first else 0,
+                                                                  _stream_ptr(stream)))
+
+
+def cp_layout(dst, src, B, S_loc, G, Hg, which, D=128, stream=None):
+    """Permute [Hg x D] blocks between the Ulysses orders (CP_* constants) through ``wan_attn_cp_layout``."""
+    import torch
+    n = B * S_loc * G * Hg * D
+    _check_plain("src", src, torch.bfloat16, n)
+    _check_plain("dst", dst, torch.bfloat16, n)
+    _check("wan_attn_cp_layout", lib().wan_attn_cp_layout(dst.data_ptr(), src.data_ptr(), B, S_loc, G, Hg, D, which,
+                                                          _stream_ptr(stream)))
 
 
 def fwd_q8_workspace_size(B, S, H, D=128) -> int:
