@@ -43,11 +43,12 @@ __global__ void __launch_bounds__(256) cp_merge_kernel(float* __restrict__ o_acc
         const bool valid = t < total;
         const long long r = valid ? (t >> 4) : 0;                    // row over [B, S, H]
         const int part = static_cast<int>(t & 15);
-        const long long h = r % H, bs = r / H, s = bs % S, b = bs / S;
-        const long long li = (b * H + h) * S + s;
-        // the row's first lane reads and updates the lse pair; its half-warp gets the weights
+        // the row's first lane reads and updates the lse pair (the only lane that needs the
+        // [B, H, S] index); its half-warp gets the weights
         float w_acc = 0.f, w_part = 1.f;
         if (valid && part == 0) {
+            const long long h = r % H, bs = r / H, s = bs % S, b = bs / S;
+            const long long li = (b * H + h) * S + s;
             const float lp = lse_part[li];
             if (first) {
                 lse_acc[li] = lp;
