@@ -120,6 +120,21 @@ def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
         cores = max(int(i.get("num_threads", 1)) for i in threadpool_info()) if threadpool_info() else 1
     except Exception:
         cores = os.cpu_count() or 1
+    if w.gemm:
+        from oracle import fp8_gemm
+        M, N, K = w.gemm
+        if x is None:
+            x = gemm_inputs(w, seed)
+        rows = synth.sample_rows(M, rows_per_head, seed=seed)
+        t0 = time.perf_counter()
+        _, xv, sx = fp8_gemm.quant_rows(x["x"][rows])        # per-token: each row on its own
+        _, wv, sw = fp8_gemm.quant_tensor(x["w"])
+        fp8_gemm.gemm_from_codes(xv, sx, wv, sw)
+        dt = time.perf_counter() - t0
+        flop = 2.0 * len(rows) * N * K
+        return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "sample": f"{len(rows)} token rows of {w.name} (quantised) against the whole quantised "
+                          f"{N} x {K} weight, fp64 numpy/BLAS, {dt:.2f} s", "_flop": flop}
     if x is None:
         x = synth.make_inputs(w, seed)
     rows = synth.sample_rows(w.S, rows_per_head, seed=seed)
@@ -129,10 +144,12 @@ def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
     flop = 4.0 * w.B * w.H * len(rows) * w.kv_len * w.D
     return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{len(rows)} query rows x {w.B * w.H} (batch, head) pairs of {w.name} "
-                      f"against all {w.kv_len} keys, fp64 numpy/BLAS, {dt:.2f} s"}
+                      f"against all {w.kv_len} keys, fp64 numpy/BLAS, {dt:.2f} s", "_flop": flop}
 
 
 def metric_of(w) -> str:
+    if w.gemm:
+        return "FP8 GEMM TFLOP/s (2*M*N*K, e4m3 x e4m3 -> fp32)"
     if w.cp:
         return f"{w.cp} context-parallel attention TFLOP/s per rank (4*B*H*S^2*D / {w.cp_ranks})"
     if w.cross:
@@ -147,6 +164,8 @@ def workload_config(w) -> dict:
         c["Skv"] = w.kv_len
     if w.cp:
         c.update(cp=w.cp, cp_ranks=w.cp_ranks, cp_note="one rank's kernels; the exchanges are not run")
+    if w.gemm:
+        c = {"workload": w.name, "M": w.gemm[0], "N": w.gemm[1], "K": w.gemm[2]}
     return c
 
 
@@ -154,13 +173,15 @@ def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    x = synth.make_inputs(w)
+    x = gemm_inputs(w, 0) if w.gemm else synth.make_inputs(w)
     rows_per_step = max(1, args.ref_rows)
     for _ in range(args.warmup):
         cpu_baseline(w, rows_per_step, x=x)
     vals = [cpu_baseline(w, rows_per_step, x=x) for _ in range(args.steps)]
     v = statistics.median(r["value"] for r in vals)
-    flop_step = 4.0 * w.B * w.H * rows_per_step * w.kv_len * w.D
+    flop_step = vals[0].pop("_flop")
+    for r in vals[1:]:
+        r.pop("_flop")
     line = {"metric": metric_of(w), "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": flop_step / (v * 1e12) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
@@ -363,6 +384,63 @@ class CpPath:
             h.copy_(d, non_blocking=True)
 
 
+class GemmPath:
+    """The FP8 linear layer: wan_fp8_quantize_rows of the bf16 activations X [M, K] (per token),
+    then wan_fp8_gemm with a weight W [N, K] quantised once beforehand (per tensor), as at
+    inference time."""
+
+    def __init__(self, wa, w, dev, x):
+        import torch
+        self.wa, self.w = wa, w
+        M, N, K = w.gemm
+
+        def pinned(bits):
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+        self.host_in = [pinned(x["x"])]
+        self.dev_in = [t.to(dev) for t in self.host_in]
+        self.w_codes, self.w_scale2 = wa.fp8_quantize_tensor(pinned(x["w"]).to(dev))
+        self.codes = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        self.scales = torch.empty(M, dtype=torch.float32, device=dev)
+        self.y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.outs = [self.y]
+        self.flop = w.fwd_flop
+        self.dominant_flop = w.fwd_flop
+        self.kernel = "wan::fp8::fp8_gemm_kernel (timed with the per-token quantiser: one FP8 linear layer)"
+        self.launches_per_step = 2
+        self.peak_key, self.dtype = "fp8", "e4m3"
+        self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.host_in)
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.host_out)
+
+    def step(self, dom_events=None):
+        wa = self.wa
+        if dom_events:
+            dom_events[0].record()
+        wa.fp8_quantize_rows(self.dev_in[0], self.codes, self.scales)
+        wa.fp8_gemm(self.codes, self.scales, self.w_codes, self.w_scale2[:1], self.y)
+        if dom_events:
+            dom_events[1].record()
+
+    def e2e_step(self):
+        self.dev_in[0].copy_(self.host_in[0], non_blocking=True)
+        self.step()
+        self.host_out[0].copy_(self.y, non_blocking=True)
+
+
+def make_path(wa, w, dev, x):
+    if w.gemm:
+        return GemmPath(wa, w, dev, x)
+    if w.cp:
+        return CpPath(wa, w, dev, x)
+    return Path(wa, w, dev, x)
+
+
+def gemm_inputs(w, seed):
+    M, N, K = w.gemm
+    return {"x": synth.make_tensor((M, K), seed, synth.STREAM_Q), "w": synth.make_tensor((N, K), seed, synth.STREAM_K)}
+
+
 def run_ours(args, w):
     import torch
     import video_dit_full_b200 as wa
@@ -381,8 +459,8 @@ def run_ours(args, w):
     wa.lib()
 
     # each rank gets its own seeded problem (seed = rank): weak scaling
-    x = synth.make_inputs(w, seed=rank)
-    path = CpPath(wa, w, dev, x) if w.cp else Path(wa, w, dev, x)
+    x = gemm_inputs(w, rank) if w.gemm else synth.make_inputs(w, seed=rank)
+    path = make_path(wa, w, dev, x)
     stream = torch.cuda.current_stream(dev)
 
     def barrier():
@@ -461,6 +539,7 @@ def run_ours(args, w):
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows, x=x)
+            line["cpu_baseline"].pop("_flop")
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

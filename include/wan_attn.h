@@ -195,6 +195,41 @@ WAN_ATTN_API int wan_attn_cp_layout(void* dst, const void* src, int B, int S_loc
                                     void* stream);
 
 /*
+ * FP8 GEMM of the DiT linear layers: the pages' FP8 GEMM (kwkr.cn Wan
+ * explainer, section 4.2: the most expensive matrix products run in FP8,
+ * weights quantised per tensor and activations per token; Wan 2.1
+ * paper-podcast summary, section "干预与形式化": FP8 GEMM, 1.13x).  For
+ * activations X [M, K] (tokens x in-features) and a weight W [N, K]
+ * (out-features x in-features, the nn.Linear layout):
+ *     sx[m] = absmax_k |X[m,k]| / 448,  xq = e4m3(x * fp32(448 / absmax))
+ *     sw    = absmax |W| / 448,         wq = e4m3(w * fp32(448 / absmax))
+ *     Y[m, n] = bf16(sx[m] * sw * sum_k xq[m,k] * wq[n,k])   (fp32 accumulation)
+ * e4m3 is the fn variant (largest finite 448), round to nearest even,
+ * saturating; the scale of an all-zero row / tensor is 1.  Codes are bytes,
+ * rows of K contiguous codes.  K must be a multiple of 16 (>= 16); every
+ * pointer 16-byte aligned unless stated; outputs overlap no input.
+ */
+/* Per-row (token) quantiser: x bf16 [M, K] -> codes u8 [M, K], scales fp32 [M]. */
+WAN_ATTN_API int wan_fp8_quantize_rows(const void* x, void* codes, float* scales, int M, int K, void* stream);
+
+/*
+ * Per-tensor quantiser: w bf16 [N, K] -> codes u8 [N, K].  scale2 points to two
+ * fp32 in device memory (8-byte aligned): on return scale2[0] = sw and
+ * scale2[1] holds absmax |W| (its bits are the kernels' scratch meanwhile).
+ */
+WAN_ATTN_API int wan_fp8_quantize_tensor(const void* w, void* codes, float* scale2, int N, int K, void* stream);
+
+/*
+ * Y = diag(a_scales) (a_codes b_codes^T) (*b_scale):
+ *   a_codes u8 [M, K], a_scales fp32 [M] (4-byte aligned), b_codes u8 [N, K],
+ *   b_scale: one fp32 in device memory (e.g. scale2 above), y bf16 [M, N].
+ *   N must be a multiple of 8; M, N >= 1; M*N < 2^40.
+ * Tensor cores: tcgen05.mma kind::f8f6f4, 128 x 256 output tiles per CTA.
+ */
+WAN_ATTN_API int wan_fp8_gemm(const void* a_codes, const float* a_scales, const void* b_codes,
+                              const float* b_scale, void* y, int M, int N, int K, void* stream);
+
+/*
  * Bytes of device workspace wan_attn_fwd_q8 needs: the quantised copies and
  * their scales, each part starting on a 256-byte boundary, in this order:
  *   int8 Q8 [B, H, S, D], int8 K8 [B, H, S, D], e4m3 V8 [B, H, S, D],

@@ -165,6 +165,7 @@ class Workload:
     Skv: int | None = None         # key/value tokens when they differ from S (cross-attention)
     cp: str | None = None          # "ring" / "ulysses": one rank's share of a G-way context split
     cp_ranks: int = 1
+    gemm: tuple | None = None      # (M, N, K) of an FP8 linear layer instead of attention
 
     @property
     def kv_len(self) -> int:
@@ -178,6 +179,9 @@ class Workload:
     def fwd_flop(self) -> float:
         """4*B*H*S*Skv*D: the forward's two S x Skv x D contractions (multiply-add = 2);
         for a context-parallel workload, one rank's 1/G share of it."""
+        if self.gemm:
+            M, N, K = self.gemm
+            return 2.0 * M * N * K
         return 4.0 * self.B * self.H * self.S * self.kv_len * self.D / self.cp_ranks
 
 
@@ -203,6 +207,11 @@ WORKLOADS = {
                                 video=(81, 720, 1280), cp="ring", cp_ranks=8),
     "ulysses8_720p_rank": Workload("ulysses8_720p_rank", 1, tokens_for_video(81, 720, 1280), 40, 128,
                                    video=(81, 720, 1280), cp="ulysses", cp_ranks=8),
+    # the DiT block's fused Q/K/V projection at 720p in FP8 (kwkr.cn Wan explainer, section 4.2):
+    # tokens x hidden (40 x 128) -> 3 x hidden
+    "fp8_qkv_720p": Workload("fp8_qkv_720p", 1, tokens_for_video(81, 720, 1280), 40, 128,
+                             video=(81, 720, 1280),
+                             gemm=(tokens_for_video(81, 720, 1280), 3 * 40 * 128, 40 * 128)),
 }
 
 

@@ -15,7 +15,7 @@ HEADER = os.path.join(ROOT, "include", "wan_attn.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(wan_attn_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(wan_\w+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")

@@ -103,6 +103,28 @@ bool make_acc_sw_map(CUtensorMap* m, void* base, int B, int S, int H) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map over an 8-bit [rows, K] matrix (K contiguous) as 2-D (K, rows), box (128, box_rows),
+// 128-byte swizzle; elements past the edges read as zero.
+bool make_rows_u8_map(CUtensorMap* m, const void* base, int rows, int K, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)K};
+    const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Shape checks of the FP8 GEMM calls: rows, K >= 1, K % 16 == 0 (16-byte code rows),
+// rows * K < 2^40.
+int check_fp8_shape(long long rows, long long K) {
+    if (rows < 1 || K < 16 || (K & 15) || rows > 0x7fffffffLL || K > 0x7fffffffLL) return WAN_ATTN_ERR_INVALID_ARG;
+    if (double(rows) * double(K) >= double(1ull << 40)) return WAN_ATTN_ERR_INVALID_ARG;
+    return WAN_ATTN_OK;
+}
+
 struct Range {
     uintptr_t lo, hi;
 };
@@ -423,6 +445,63 @@ int wan_attn_cp_layout(void* dst, const void* src, int B, int S_loc, int G, int 
     return launch_cp_layout(dst, src, B, S_loc, G, Hg * D * 2 / 16, which, static_cast<cudaStream_t>(stream)) == 0
                ? WAN_ATTN_OK
                : WAN_ATTN_ERR_CUDA;
+}
+
+int wan_fp8_quantize_rows(const void* x, void* codes, float* scales, int M, int K, void* stream) {
+    if (!x || !codes || !scales) return WAN_ATTN_ERR_INVALID_ARG;
+    const int st = check_fp8_shape(M, K);
+    if (st != WAN_ATTN_OK) return st;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return WAN_ATTN_ERR_INVALID_ARG;
+    const size_t n = size_t(M) * K;
+    const Range rx = range_of(x, n * 2), rc = range_of(codes, n), rs = range_of(scales, size_t(M) * 4);
+    if (overlaps(rx, rc) || overlaps(rx, rs) || overlaps(rc, rs)) return WAN_ATTN_ERR_INVALID_ARG;
+    return launch_fp8_quant_rows(x, codes, scales, M, K, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                               : WAN_ATTN_ERR_CUDA;
+}
+
+int wan_fp8_quantize_tensor(const void* w, void* codes, float* scale2, int N, int K, void* stream) {
+    if (!w || !codes || !scale2) return WAN_ATTN_ERR_INVALID_ARG;
+    const int st = check_fp8_shape(N, K);
+    if (st != WAN_ATTN_OK) return st;
+    if (!aligned16(w) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scale2) & 7u))
+        return WAN_ATTN_ERR_INVALID_ARG;
+    const size_t n = size_t(N) * K;
+    const Range rw = range_of(w, n * 2), rc = range_of(codes, n), rs = range_of(scale2, 8);
+    if (overlaps(rw, rc) || overlaps(rw, rs) || overlaps(rc, rs)) return WAN_ATTN_ERR_INVALID_ARG;
+    return launch_fp8_quant_tensor(w, codes, scale2, static_cast<long long>(n), static_cast<cudaStream_t>(stream)) == 0
+               ? WAN_ATTN_OK
+               : WAN_ATTN_ERR_CUDA;
+}
+
+int wan_fp8_gemm(const void* a_codes, const float* a_scales, const void* b_codes, const float* b_scale, void* y,
+                 int M, int N, int K, void* stream) {
+    if (!a_codes || !a_scales || !b_codes || !b_scale || !y) return WAN_ATTN_ERR_INVALID_ARG;
+    int st = check_fp8_shape(M, K);
+    if (st == WAN_ATTN_OK) st = check_fp8_shape(N, K);
+    if (st != WAN_ATTN_OK) return st;
+    if ((N & 7) || double(M) * N >= double(1ull << 40)) return WAN_ATTN_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(y) || (reinterpret_cast<uintptr_t>(a_scales) & 3u) ||
+        (reinterpret_cast<uintptr_t>(b_scale) & 3u))
+        return WAN_ATTN_ERR_INVALID_ARG;
+    const Range ry = range_of(y, size_t(M) * N * 2);
+    const Range ins[] = {range_of(a_codes, size_t(M) * K), range_of(a_scales, size_t(M) * 4),
+                         range_of(b_codes, size_t(N) * K), range_of(b_scale, 4)};
+    for (const Range& in : ins)
+        if (overlaps(ry, in)) return WAN_ATTN_ERR_INVALID_ARG;
+    CUtensorMap ta, tb;
+    if (!make_rows_u8_map(&ta, a_codes, M, K, 128) || !make_rows_u8_map(&tb, b_codes, N, K, 256))
+        return WAN_ATTN_ERR_CUDA;
+    Fp8GemmParams p;
+    p.a_scales = a_scales;
+    p.b_scale = b_scale;
+    p.y = y;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.wait_budget_ns = wait_budget_ns();
+    p.status = device_status_word();
+    if (!p.status) return WAN_ATTN_ERR_CUDA;
+    return launch_fp8_gemm(ta, tb, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
 }
 
 int wan_attn_sync_status(void* stream) {

@@ -33,11 +33,6 @@ namespace q8 {
 constexpr int BLK = 64;          // quantisation block (tokens)
 constexpr int HD = 128;
 
-__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
-}
 
 // one CTA per (tensor, b*H + h, 64-token block), flattened into blockIdx.x in that order;
 // 256 threads: thread = (token row of the block, quarter of D)

@@ -53,6 +53,15 @@ struct Q8AttnParams {
     int* status;
 };
 
+struct Fp8GemmParams {
+    const float* a_scales;            // fp32 [M]: per-row (token) scales of the activation codes
+    const float* b_scale;             // fp32 [1]: the weight's per-tensor scale (device memory)
+    void* y;                          // bf16 [M, N]
+    int M, N, K;
+    unsigned long long wait_budget_ns;
+    int* status;
+};
+
 // Device address of the status word on the current device (nullptr on failure).
 int* device_status_word();
 unsigned long long wait_budget_ns();
@@ -75,6 +84,11 @@ int launch_cp_merge(float* o_acc, float* lse_acc, const void* o_part, const floa
                     int S, int H, int first, cudaStream_t stream);
 int launch_cp_accumulate(float* acc, const void* part, void* out, long long n8, int first, cudaStream_t stream);
 int launch_cp_layout(void* dst, const void* src, int B, int S, int G, int blk16, int which, cudaStream_t stream);
+
+// FP8 GEMM of the linear layers (fp8_gemm.cu).  0 on success.
+int launch_fp8_quant_rows(const void* x, void* codes, float* scales, int M, int K, cudaStream_t stream);
+int launch_fp8_quant_tensor(const void* w, void* codes, float* scale2, long long n, cudaStream_t stream);
+int launch_fp8_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const Fp8GemmParams& p, cudaStream_t stream);
 
 int launch_q8(const Q8QuantParams& qp, const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv8,
               const Q8AttnParams& p, cudaStream_t stream);

@@ -29,6 +29,9 @@ SIGNATURES = [
     ("wan_attn_cp_merge", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     ("wan_attn_cp_accumulate", _I, [_P, _P, _P, _Z, _I, _P]),
     ("wan_attn_cp_layout", _I, [_P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    ("wan_fp8_quantize_rows", _I, [_P, _P, _P, _I, _I, _P]),
+    ("wan_fp8_quantize_tensor", _I, [_P, _P, _P, _I, _I, _P]),
+    ("wan_fp8_gemm", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     ("wan_attn_fwd_q8_workspace_size", _Z, [_I, _I, _I, _I]),
     ("wan_attn_fwd_q8", _I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P, _Z, _P]),
     ("wan_attn_bwd_noalloc", _I, [_P, _P, _P, _P, _P, _F, _P, _P, _P, _I, _I, _I, _I, _P]),
@@ -242,6 +245,63 @@ def cp_layout(dst, src, B, S_loc, G, Hg, which, D=128, stream=None):
     _check_plain("dst", dst, torch.bfloat16, n)
     _check("wan_attn_cp_layout", lib().wan_attn_cp_layout(dst.data_ptr(), src.data_ptr(), B, S_loc, G, Hg, D, which,
                                                           _stream_ptr(stream)))
+
+
+def fp8_quantize_rows(x, codes=None, scales=None, stream=None):
+    """Per-token e4m3 codes (uint8 [M, K]) and fp32 scales [M] of bf16 x [M, K] (``wan_fp8_quantize_rows``)."""
+    import torch
+    _check_plain("x", x, torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be [M, K]")
+    M, K = x.shape
+    codes = torch.empty((M, K), dtype=torch.uint8, device=x.device) if codes is None else codes
+    scales = torch.empty(M, dtype=torch.float32, device=x.device) if scales is None else scales
+    _check_plain("codes", codes, torch.uint8, M * K)
+    _check_plain("scales", scales, torch.float32, M)
+    _check("wan_fp8_quantize_rows", lib().wan_fp8_quantize_rows(x.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                                                                M, K, _stream_ptr(stream)))
+    return codes, scales
+
+
+def fp8_quantize_tensor(w, codes=None, scale2=None, stream=None):
+    """Per-tensor e4m3 codes (uint8 [N, K]) of bf16 w [N, K]; scale2 fp32 [2] = (sw, absmax)."""
+    import torch
+    _check_plain("w", w, torch.bfloat16)
+    if w.dim() != 2:
+        raise ValueError("w must be [N, K]")
+    N, K = w.shape
+    codes = torch.empty((N, K), dtype=torch.uint8, device=w.device) if codes is None else codes
+    scale2 = torch.empty(2, dtype=torch.float32, device=w.device) if scale2 is None else scale2
+    _check_plain("codes", codes, torch.uint8, N * K)
+    _check_plain("scale2", scale2, torch.float32, 2)
+    _check("wan_fp8_quantize_tensor", lib().wan_fp8_quantize_tensor(w.data_ptr(), codes.data_ptr(),
+                                                                    scale2.data_ptr(), N, K, _stream_ptr(stream)))
+    return codes, scale2
+
+
+def fp8_gemm(a_codes, a_scales, b_codes, b_scale, y=None, stream=None):
+    """bf16 Y [M, N] = diag(a_scales) (a_codes b_codes^T) b_scale[0] through ``wan_fp8_gemm``."""
+    import torch
+    _check_plain("a_codes", a_codes, torch.uint8)
+    _check_plain("b_codes", b_codes, torch.uint8)
+    if a_codes.dim() != 2 or b_codes.dim() != 2 or a_codes.shape[1] != b_codes.shape[1]:
+        raise ValueError("a_codes [M, K] and b_codes [N, K] must share K")
+    M, K = a_codes.shape
+    N = b_codes.shape[0]
+    _check_plain("a_scales", a_scales, torch.float32, M)
+    _check_plain("b_scale", b_scale, torch.float32)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device) if y is None else y
+    _check_plain("y", y, torch.bfloat16, M * N)
+    _check("wan_fp8_gemm", lib().wan_fp8_gemm(a_codes.data_ptr(), a_scales.data_ptr(), b_codes.data_ptr(),
+                                              b_scale.data_ptr(), y.data_ptr(), M, N, K, _stream_ptr(stream)))
+    return y
+
+
+def fp8_linear(x, w_codes, w_scale, stream=None):
+    """Y = the FP8 linear layer of bf16 activations x [M, K] with a weight already quantised
+    by fp8_quantize_tensor: the per-token quantiser, then the GEMM."""
+    codes, scales = fp8_quantize_rows(x, stream=stream)
+    return fp8_gemm(codes, scales, w_codes, w_scale, stream=stream)
 
 
 def fwd_q8_workspace_size(B, S, H, D=128) -> int:
