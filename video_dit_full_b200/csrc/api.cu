@@ -488,8 +488,9 @@ int wan_fp8_gemm(const void* a_codes, const float* a_scales, const void* b_codes
                          range_of(b_codes, size_t(N) * K), range_of(b_scale, 4)};
     for (const Range& in : ins)
         if (overlaps(ry, in)) return WAN_ATTN_ERR_INVALID_ARG;
-    CUtensorMap ta, tb;
-    if (!make_rows_u8_map(&ta, a_codes, M, K, 128) || !make_rows_u8_map(&tb, b_codes, N, K, 256))
+    CUtensorMap ta, tb, tb_half;
+    if (!make_rows_u8_map(&ta, a_codes, M, K, 128) || !make_rows_u8_map(&tb, b_codes, N, K, 256) ||
+        !make_rows_u8_map(&tb_half, b_codes, N, K, 128))
         return WAN_ATTN_ERR_CUDA;
     Fp8GemmParams p;
     p.a_scales = a_scales;
@@ -501,7 +502,8 @@ int wan_fp8_gemm(const void* a_codes, const float* a_scales, const void* b_codes
     p.wait_budget_ns = wait_budget_ns();
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
-    return launch_fp8_gemm(ta, tb, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
+    return launch_fp8_gemm(ta, tb, tb_half, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                     : WAN_ATTN_ERR_CUDA;
 }
 
 int wan_attn_sync_status(void* stream) {

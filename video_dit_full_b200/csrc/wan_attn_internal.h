@@ -88,7 +88,9 @@ int launch_cp_layout(void* dst, const void* src, int B, int S, int G, int blk16,
 // FP8 GEMM of the linear layers (fp8_gemm.cu).  0 on success.
 int launch_fp8_quant_rows(const void* x, void* codes, float* scales, int M, int K, cudaStream_t stream);
 int launch_fp8_quant_tensor(const void* w, void* codes, float* scale2, long long n, cudaStream_t stream);
-int launch_fp8_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const Fp8GemmParams& p, cudaStream_t stream);
+// tb: W's map with 256-row boxes (1-CTA kernel); tb_half: 128-row boxes (CTA pairs).
+int launch_fp8_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb_half, const Fp8GemmParams& p,
+                    cudaStream_t stream);
 
 int launch_q8(const Q8QuantParams& qp, const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv8,
               const Q8AttnParams& p, cudaStream_t stream);
