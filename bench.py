@@ -33,7 +33,7 @@ METRIC = "attention TFLOP/s (4*B*H*S^2*D fwd)"
 
 # DRAM bytes (read + write) of one launch of the dominant kernel from an ncu
 # capture (profiles/), per workload; None where the kernel changed since.
-TRAFFIC = {"wan14b_720p": 3.335e9, "train_480p_fwd_bwd": 3.54e9, "q8_720p": 1.934e9}
+TRAFFIC = {"wan14b_720p": 3.335e9, "train_480p_fwd_bwd": 3.54e9, "q8_720p": 1.934e9, "fp8_qkv_720p": 5.028e9}
 
 
 def load_peaks():
@@ -406,7 +406,7 @@ class GemmPath:
         self.outs = [self.y]
         self.flop = w.fwd_flop
         self.dominant_flop = w.fwd_flop
-        self.kernel = "wan::fp8::fp8_gemm_kernel (timed with the per-token quantiser: one FP8 linear layer)"
+        self.kernel = "wan::fp8::fp8_gemm_pair_kernel (timed with the per-token quantiser: one FP8 linear layer)"
         self.launches_per_step = 2
         self.peak_key, self.dtype = "fp8", "e4m3"
         self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
@@ -563,7 +563,9 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if args.S or args.H:
         import dataclasses
-        w = dataclasses.replace(w, S=args.S or w.S, H=args.H or w.H, name=f"{w.name}@S{args.S or w.S}H{args.H or w.H}")
+        gemm = (args.S or w.gemm[0],) + tuple(w.gemm[1:]) if w.gemm else None   # --S sets a GEMM's M
+        w = dataclasses.replace(w, S=args.S or w.S, H=args.H or w.H, gemm=gemm,
+                                name=f"{w.name}@S{args.S or w.S}H{args.H or w.H}")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -9,8 +9,9 @@
 //                      sx = absmax / 448, codes = e4m3(fp32(x * fp32(448 / absmax))).
 //   fp8_absmax /       W [N, K] bf16 -> its absmax (atomic max of the bit patterns of
 //   fp8_quant_tensor   non-negative floats), then e4m3 codes with the one per-tensor scale.
-//   fp8_gemm_kernel    persistent, one CTA per SM walking 128 x 256 output tiles (N fastest,
-//                      so a row block of X and all of W stay in L2):
+//   fp8_gemm_kernel    persistent, one CTA per SM walking 128 x 256 output tiles (in groups of
+//                      16 row blocks, the row block fastest, so the tiles in flight share
+//                      a few row blocks of X and column blocks of W in L2):
 //                        warp 0      TMA: [128 x 128 B] of X and [256 x 128 B] of W per stage,
 //                                    4 stages, 128-byte swizzle, zero fill past the edges
 //                        warp 1      tcgen05.mma kind::f8f6f4 (e4m3 x e4m3 -> fp32), M128 N256
@@ -137,6 +138,22 @@ constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
 constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
 constexpr int NTHREADS = 192;                       // warp 0 TMA, 1 MMA, 2-5 epilogue
 constexpr uint32_t TMEM_COLS = 512;                 // two 256-column fp32 accumulators
+#ifndef FP8_GROUP_M
+#define FP8_GROUP_M 16
+#endif
+constexpr int GROUP_M = FP8_GROUP_M;                // tile order: row blocks in groups of GROUP_M
+
+// Tile t -> (row block, column block): the tiles are walked in groups of GROUP_M row blocks,
+// the row block varying fastest inside a group.  The CTAs at work at any moment then share a
+// few row blocks of X and a few column blocks of W, which stay in L2.
+__device__ __forceinline__ void tile_of(long long t, int m_tiles, int n_tiles, int& mb, int& nb) {
+    const long long per_group = static_cast<long long>(GROUP_M) * n_tiles;
+    const int g = static_cast<int>(t / per_group);
+    const int rows = min(GROUP_M, m_tiles - g * GROUP_M);
+    const long long w = t - g * per_group;
+    mb = g * GROUP_M + static_cast<int>(w % rows);
+    nb = static_cast<int>(w / rows);
+}
 
 __global__ void __launch_bounds__(NTHREADS, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
@@ -187,7 +204,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
             long long it = 0;
             bool ok = true;
             for (long long t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-                const int m0 = static_cast<int>(t / n_tiles) * BM, n0 = static_cast<int>(t % n_tiles) * BN;
+                int mb, nbk;
+                tile_of(t, m_tiles, n_tiles, mb, nbk);
+                const int m0 = mb * BM, n0 = nbk * BN;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = static_cast<int>(it % STAGES);
                     const int use = static_cast<int>((it / STAGES) & 1);
@@ -243,7 +262,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
         int tc = 0;
         bool ok = true;
         for (long long t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
-            const int m0 = static_cast<int>(t / n_tiles) * BM, n0 = static_cast<int>(t % n_tiles) * BN;
+            int mb, nbk;
+            tile_of(t, m_tiles, n_tiles, mb, nbk);
+            const int m0 = mb * BM, n0 = nbk * BN;
             const int b = tc & 1;
             ok = wait_warp(bar(TFULL + b), (tc >> 1) & 1, wc);
             if (!ok) break;
@@ -395,8 +416,10 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_con
             long long it = 0;
             bool ok = true;
             for (long long t = pair; t < tiles && ok; t += npairs) {
-                const int m0 = static_cast<int>(t / n_tiles) * 256 + static_cast<int>(rank) * 128;
-                const int nb = static_cast<int>(t % n_tiles) * BN + static_cast<int>(rank) * 128;
+                int mb, nbk;
+                tile_of(t, m_tiles, n_tiles, mb, nbk);
+                const int m0 = mb * 256 + static_cast<int>(rank) * 128;
+                const int nb = nbk * BN + static_cast<int>(rank) * 128;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const int s = static_cast<int>(it % STAGES2);
                     const int use = static_cast<int>((it / STAGES2) & 1);
@@ -456,8 +479,10 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_con
         int tc = 0;
         bool ok = true;
         for (long long t = pair; t < tiles && ok; t += npairs, ++tc) {
-            const int m0 = static_cast<int>(t / n_tiles) * 256 + static_cast<int>(rank) * 128;
-            const int n0 = static_cast<int>(t % n_tiles) * BN;
+            int mb, nbk;
+            tile_of(t, m_tiles, n_tiles, mb, nbk);
+            const int m0 = mb * 256 + static_cast<int>(rank) * 128;
+            const int n0 = nbk * BN;
             const int b = tc & 1;
             ok = wait_warp(bar(TF2 + b), (tc >> 1) & 1, wc);
             if (!ok) break;
