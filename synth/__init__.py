@@ -6,7 +6,7 @@ describes the workloads' shapes.  Both the oracle and the GPU path read the
 same host bytes that it writes.
 
 Streams: 0 = Q, 1 = K, 2 = V, 3 = dO, 4 = peaky-head choice,
-5 = sampled query rows, 6 = sampled key rows.
+5 = sampled query rows, 6 = sampled key rows, 7 = block-sparse masks.
 """
 from __future__ import annotations
 
@@ -24,6 +24,7 @@ _lib = None
 
 STREAM_Q, STREAM_K, STREAM_V, STREAM_DO = 0, 1, 2, 3
 STREAM_PEAKY, STREAM_QROWS, STREAM_KROWS = 4, 5, 6
+STREAM_MASK = 7
 
 
 def build(force: bool = False) -> str:
@@ -233,6 +234,17 @@ def sample_rows(S: int, n: int = 256, seed: int = 0, stream: int = STREAM_QROWS)
     u = uniform(seed, stream, S)[1:S - 1]
     pick = np.argsort(u, kind="stable")[: n - 2] + 1
     return np.sort(np.concatenate([[0, S - 1], pick]).astype(np.int64))
+
+
+def block_mask(B: int, H: int, nqb: int, nkb: int, keep: float, seed: int = 0) -> np.ndarray:
+    """A 64 x 64 block mask uint8 [B, H, nqb, nkb] keeping max(1, round(keep * nkb)) key blocks
+    per query block: those with the smallest uniform draws of stream 7 (row-major order)."""
+    u = uniform(seed, STREAM_MASK, B * H * nqb * nkb).reshape(B, H, nqb, nkb)
+    n = max(1, int(round(keep * nkb)))
+    pick = np.argsort(u, axis=3, kind="stable")[..., :n]
+    mask = np.zeros((B, H, nqb, nkb), dtype=np.uint8)
+    np.put_along_axis(mask, pick, 1, axis=3)
+    return mask
 
 
 def make_tensor(shape, seed: int, stream: int, nthreads=None) -> np.ndarray:
