@@ -135,6 +135,21 @@ def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
         return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                 "sample": f"{len(rows)} token rows of {w.name} (quantised) against the whole quantised "
                           f"{N} x {K} weight, fp64 numpy/BLAS, {dt:.2f} s", "_flop": flop}
+    if w.sparse_keep:
+        from oracle import block_sparse
+        if x is None:
+            x = synth.make_inputs(w, seed)
+        nb = (w.S + 63) // 64
+        mask = synth.block_mask(w.B, w.H, nb, nb, w.sparse_keep, seed=seed)
+        rows = synth.sample_rows(w.S, rows_per_head, seed=seed)
+        size = np.minimum(64, w.S - 64 * np.arange(nb)).astype(np.float64)
+        t0 = time.perf_counter()
+        block_sparse.attn_fwd_block_sparse(x["q"], x["k"], x["v"], mask, rows=rows)
+        dt = time.perf_counter() - t0
+        flop = float(4.0 * w.D * (mask[:, :, rows // 64, :].astype(np.float64) @ size).sum())
+        return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "sample": f"{len(rows)} query rows x {w.B * w.H} (batch, head) pairs of {w.name} against "
+                          f"their allowed key blocks (fp64, masked dense rows), {dt:.2f} s", "_flop": flop}
     if x is None:
         x = synth.make_inputs(w, seed)
     rows = synth.sample_rows(w.S, rows_per_head, seed=seed)
@@ -148,6 +163,8 @@ def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
 
 
 def metric_of(w) -> str:
+    if w.sparse_keep:
+        return "block-sparse attention TFLOP/s (4*D*64*64 per allowed 64x64 block)"
     if w.gemm:
         return "FP8 GEMM TFLOP/s (2*M*N*K, e4m3 x e4m3 -> fp32)"
     if w.cp:
@@ -428,7 +445,64 @@ class GemmPath:
         self.host_out[0].copy_(self.y, non_blocking=True)
 
 
+class SparsePath:
+    """Block-sparse attention: one wan_attn_fwd_block_sparse over a seeded 64 x 64 block mask.
+    `flop` counts only the allowed blocks (4 * D * |query block| * |key block| each); the
+    dense-equivalent count and the fraction of key blocks the CTAs' unions cover are reported
+    beside it."""
+
+    def __init__(self, wa, w, dev, x):
+        import torch
+        self.wa, self.w = wa, w
+        shape = (w.B, w.S, w.H, w.D)
+
+        def pinned(bits):
+            return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+        nb = (w.S + 63) // 64
+        self.mask_host = synth.block_mask(w.B, w.H, nb, nb, w.sparse_keep, seed=x["seed"])
+        size = np.minimum(64, w.S - 64 * np.arange(nb)).astype(np.float64)
+        self.flop = float(4.0 * w.D * np.einsum("bhij,i,j->", self.mask_host.astype(np.float64), size, size))
+        self.dense_flop = w.fwd_flop
+        m4 = np.pad(self.mask_host, ((0, 0), (0, 0), (0, (-nb) % 4), (0, 0)))
+        union = m4.reshape(w.B, w.H, -1, 4, nb).max(axis=3)
+        self.union_frac = float(union.mean())
+        self.host_in = [pinned(x[n]) for n in ("q", "k", "v")]
+        self.dev_in = [t.to(dev) for t in self.host_in]
+        self.mask = torch.from_numpy(self.mask_host).to(dev)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty(shape, **bf)
+        self.lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(wa.block_sparse_workspace_size(w.B, w.S, w.S, w.H, w.D), dtype=torch.uint8,
+                              device=dev)
+        self.outs = [self.o, self.lse]
+        self.dominant_flop = self.flop
+        self.kernel = "wan::fwd::attn_fwd_kernel<true> (with its key-block list kernel: one wan_attn_fwd_block_sparse)"
+        self.launches_per_step = 2
+        self.peak_key, self.dtype = "bf16", "bf16"
+        self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.host_in)
+        self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.host_out)
+
+    def step(self, dom_events=None):
+        if dom_events:
+            dom_events[0].record()
+        q, k, v = self.dev_in
+        self.wa.fwd_block_sparse(q, k, v, self.mask, self.o, self.lse, workspace=self.ws)
+        if dom_events:
+            dom_events[1].record()
+
+    def e2e_step(self):
+        for d, h in zip(self.dev_in, self.host_in):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        for h, d in zip(self.host_out, self.outs):
+            h.copy_(d, non_blocking=True)
+
+
 def make_path(wa, w, dev, x):
+    if w.sparse_keep:
+        return SparsePath(wa, w, dev, x)
     if w.gemm:
         return GemmPath(wa, w, dev, x)
     if w.cp:
@@ -460,6 +534,7 @@ def run_ours(args, w):
 
     # each rank gets its own seeded problem (seed = rank): weak scaling
     x = gemm_inputs(w, rank) if w.gemm else synth.make_inputs(w, seed=rank)
+    x["seed"] = rank
     path = make_path(wa, w, dev, x)
     stream = torch.cuda.current_stream(dev)
 
@@ -527,6 +602,9 @@ def run_ours(args, w):
                        "flop_per_step": path.flop, "parallelism": f"replicas{world}",
                        "l2": "inputs (%.2f GB) exceed the 126 MB L2; no flush" % in_gb},
             "gpu_launches": args.steps * path.launches_per_step,
+            **({"sparse": {"keep": w.sparse_keep, "union_fraction_computed": path.union_frac,
+                           "dense_equivalent_tflops": whole_job_tflops(world, path.dense_flop, args.steps, total_ms)}}
+               if w.sparse_keep else {}),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": TRAFFIC.get(w.name),
                          "peak_source": peak_src, "frac_of_sustained": achieved / sustained,

@@ -141,6 +141,34 @@ WAN_ATTN_API int wan_attn_cross_bwd(const void* q, const void* k, const void* v,
                                     int H, int D, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Block-sparse forward with a given 64 x 64 block mask: the block-sparse
+ * attention of the FastWan / VSA article on the first page ("一夜颠覆Sora神话，
+ * H200单卡5秒出片…": each 64-token query block keeps a subset of the 64-token
+ * key blocks, 87.5 % sparsity in its runs; FlexAttention compared on the same
+ * 64 x 64 block-sparse mask).  The mask is an input (the learned coarse stage
+ * that chooses blocks is not part of this library).  Block i of a sequence
+ * holds tokens [64 i, 64 i + 64), the last block possibly short.
+ *   q : bf16 [B, Sq, H, D];  k, v : bf16 [B, Skv, H, D];  D must be 128
+ *   block_mask : uint8 [B, H, ceil(Sq/64), ceil(Skv/64)], non-zero = query block
+ *                i attends key block j (no alignment needed)
+ *   o : out bf16 [B, Sq, H, D];  lse : out fp32 [B, H, Sq]
+ *   A row whose query block attends no key block gets o = 0 and lse = -inf.
+ *   workspace, workspace_bytes : caller-owned device memory, 256-byte aligned,
+ *     at least wan_attn_fwd_block_sparse_workspace_size bytes: the per-CTA
+ *     lists of attended key blocks (int32 [B, H, ceil(Sq/256), ceil(Skv/64)])
+ *     and their lengths, built on the device by this call.
+ * Work: a CTA covers 256 queries (4 query blocks) and runs its 128-row MMAs
+ * over the union of the key blocks its 4 query blocks attend, two blocks per
+ * step; the softmax masks each row to its own blocks.  With an all-ones mask
+ * the result equals wan_attn_fwd bit for bit.  Other conventions as
+ * wan_attn_fwd.
+ */
+WAN_ATTN_API size_t wan_attn_fwd_block_sparse_workspace_size(int B, int Sq, int Skv, int H, int D);
+WAN_ATTN_API int wan_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                                           const uint8_t* block_mask, int B, int Sq, int Skv, int H, int D,
+                                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Context parallelism: the building blocks of the two schemes the pages name for
  * sequences too long for one GPU (kwkr.cn Wan explainer, section 3.2: the token
  * sequence is split over GPUs and combined with Ulysses and Ring Attention;

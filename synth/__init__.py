@@ -167,6 +167,7 @@ class Workload:
     cp: str | None = None          # "ring" / "ulysses": one rank's share of a G-way context split
     cp_ranks: int = 1
     gemm: tuple | None = None      # (M, N, K) of an FP8 linear layer instead of attention
+    sparse_keep: float = 0.0       # block-sparse: fraction of 64-token key blocks each query block keeps
 
     @property
     def kv_len(self) -> int:
@@ -208,6 +209,10 @@ WORKLOADS = {
                                 video=(81, 720, 1280), cp="ring", cp_ranks=8),
     "ulysses8_720p_rank": Workload("ulysses8_720p_rank", 1, tokens_for_video(81, 720, 1280), 40, 128,
                                    video=(81, 720, 1280), cp="ulysses", cp_ranks=8),
+    # block-sparse attention keeping 1/8 of the 64 x 64 blocks (87.5 % sparsity, the FastWan /
+    # VSA article on the first page), random seeded mask
+    "sparse8_720p": Workload("sparse8_720p", 1, tokens_for_video(81, 720, 1280), 40, 128,
+                             video=(81, 720, 1280), sparse_keep=0.125),
     # the DiT block's fused Q/K/V projection at 720p in FP8 (kwkr.cn Wan explainer, section 4.2):
     # tokens x hidden (40 x 128) -> 3 x hidden
     "fp8_qkv_720p": Workload("fp8_qkv_720p", 1, tokens_for_video(81, 720, 1280), 40, 128,

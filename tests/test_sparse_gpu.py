@@ -1,0 +1,94 @@
+"""Parity of the block-sparse forward (wan_attn_fwd_block_sparse, through the C ABI) with the oracle
+(oracle/block_sparse.py): the bf16 forward's bars (O max-abs 1e-2 and rel-Frobenius 5e-3, LSE
+1e-3) on the rows that attend something; rows that attend nothing must be exactly O = 0,
+LSE = -inf.  An all-ones mask must reproduce wan_attn_fwd bit for bit (same arithmetic)."""
+import numpy as np
+import pytest
+
+import synth
+from gpu_util import bf16_to_f64, errors, inputs_for_cross, to_device
+from oracle import block_sparse as bs
+
+pytestmark = pytest.mark.gpu
+
+O_MAX_ABS, O_REL_FROB, LSE_MAX_ABS = 1e-2, 5e-3, 1e-3
+
+
+def run(x, mask):
+    import torch
+    import video_dit_full_b200 as wa
+    q, k, v = (to_device(x[n]) for n in "qkv")
+    m = torch.from_numpy(np.ascontiguousarray(mask)).cuda()
+    o, lse = wa.fwd_block_sparse(q, k, v, m)
+    wa.check_status()
+    return o, lse
+
+
+def check(x, mask, rows=None, heads=None):
+    o, lse = run(x, mask)
+    want_o, want_lse = bs.attn_fwd_block_sparse(x["q"], x["k"], x["v"], mask, rows=rows, heads=heads)
+    got_o, got_lse = bf16_to_f64(o), lse.cpu().numpy().astype(np.float64)
+    if rows is not None:
+        got_o, got_lse = got_o[:, rows], got_lse[:, :, rows]
+    if heads is not None:
+        got_o, got_lse = got_o[:, :, heads], got_lse[:, heads]
+    empty = np.isneginf(want_lse)                                    # [B, H, R]
+    assert np.all(np.isneginf(got_lse[empty]))
+    assert np.all(got_o.transpose(0, 2, 1, 3)[empty] == 0)
+    live = ~empty
+    go, wo = got_o.transpose(0, 2, 1, 3)[live], want_o.transpose(0, 2, 1, 3)[live]
+    if go.size:
+        max_abs, rel = errors(go, wo)
+        lse_err = float(np.abs(got_lse[live] - want_lse[live]).max())
+        print(f"O max-abs {max_abs:.3e} rel-frob {rel:.3e}  LSE max-abs {lse_err:.3e}  empty rows {empty.sum()}")
+        assert max_abs <= O_MAX_ABS and rel <= O_REL_FROB, (max_abs, rel)
+        assert lse_err <= LSE_MAX_ABS, lse_err
+
+
+def test_all_ones_mask_is_the_dense_call_bit_for_bit():
+    import torch
+    import video_dit_full_b200 as wa
+    x = inputs_for_cross(2, 1000, 1000, 3, seed=21)
+    mask = np.ones((2, 3, bs.blocks(1000), bs.blocks(1000)), dtype=np.uint8)
+    o, lse = run(x, mask)
+    q, k, v = (to_device(x[n]) for n in "qkv")
+    od, ld = wa.fwd(q, k, v)
+    wa.check_status()
+    assert torch.equal(o, od) and torch.equal(lse, ld)
+
+
+@pytest.mark.parametrize("Sq,Skv,keep", [(1000, 1000, 0.5), (1000, 1000, 0.125), (300, 777, 0.25),
+                                         (4100, 4100, 0.125), (65, 64, 1.0)])
+def test_random_masks(Sq, Skv, keep):
+    B, H = 1, 2
+    x = inputs_for_cross(B, Sq, Skv, H, seed=Sq + Skv)
+    mask = synth.block_mask(B, H, bs.blocks(Sq), bs.blocks(Skv), keep, seed=Sq)
+    check(x, mask)
+
+
+def test_rows_and_ctas_that_attend_nothing():
+    B, H, S = 1, 2, 1300
+    x = inputs_for_cross(B, S, S, H, seed=4)
+    mask = synth.block_mask(B, H, bs.blocks(S), bs.blocks(S), 0.3, seed=4)
+    mask[0, 0, 1] = 0                     # one query block of head 0
+    mask[0, 1, 4:8] = 0                   # every query block of CTA 1 (tokens 256-511) of head 1
+    mask[0, 1, 20] = 0                    # the short last block
+    check(x, mask)
+
+
+def test_block_diagonal_mask():
+    B, H, S = 1, 2, 777
+    x = inputs_for_cross(B, S, S, H, seed=5)
+    nb = bs.blocks(S)
+    mask = np.zeros((B, H, nb, nb), dtype=np.uint8)
+    for i in range(nb):
+        mask[:, :, i, i] = 1
+    check(x, mask)
+
+
+def test_720p_at_one_eighth_density_sampled_rows():
+    w = synth.WORKLOADS["wan14b_720p"]
+    x = synth.make_inputs(w)
+    nb = bs.blocks(w.S)
+    mask = synth.block_mask(w.B, w.H, nb, nb, 0.125, seed=0)
+    check(x, mask, rows=synth.sample_rows(w.S, 256))

@@ -207,7 +207,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     if (!make_bshd_map(&tq, q, B, Sq, H, D, 128) || !make_bshd_map(&tk, k, B, Skv, H, D, 128) ||
         !make_bshd_map(&tv, v, B, Skv, H, D, 128))
         return WAN_ATTN_ERR_CUDA;
-    FwdParams p;
+    FwdParams p{};
     p.o = o;
     p.lse = lse;
     p.B = B;
@@ -219,6 +219,63 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
     return launch_fwd(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
+}
+
+// Block-sparse forward: per CTA (2 Q tiles = 4 query blocks of 64) the list of attended key
+// blocks, int32 [B, H, nctas, nkb], then the lists' lengths [B, H, nctas].
+size_t sparse_ws_size(int B, int Sq, int Skv, int H, int D) {
+    if (check_shape(B, Sq, H, D) != WAN_ATTN_OK || check_shape(B, Skv, H, D) != WAN_ATTN_OK) return 0;
+    const size_t nctas = (size_t(Sq) + 255) / 256, nkb = (size_t(Skv) + 63) / 64;
+    return align256(size_t(B) * H * nctas * nkb * 4) + align256(size_t(B) * H * nctas * 4);
+}
+
+int fwd_block_sparse_impl(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* mask,
+                          int B, int Sq, int Skv, int H, int D, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    if (!q || !k || !v || !o || !lse || !mask) return WAN_ATTN_ERR_INVALID_ARG;
+    int st = check_shape(B, Sq, H, D);
+    if (st == WAN_ATTN_OK) st = check_shape(B, Skv, H, D);
+    if (st != WAN_ATTN_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return WAN_ATTN_ERR_INVALID_ARG;
+    const size_t need = sparse_ws_size(B, Sq, Skv, H, D);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return WAN_ATTN_ERR_WORKSPACE;
+    const int nqb = (Sq + 63) / 64, nkb = (Skv + 63) / 64, nctas = (Sq + 255) / 256;
+    const size_t nq = size_t(B) * Sq * H * D, nkv = size_t(B) * Skv * H * D;
+    const Range ins[] = {range_of(q, nq * 2), range_of(k, nkv * 2), range_of(v, nkv * 2),
+                         range_of(mask, size_t(B) * H * nqb * nkb)};
+    const Range outs[] = {range_of(o, nq * 2), range_of(lse, size_t(B) * H * Sq * 4), range_of(workspace, need)};
+    for (size_t a = 0; a < 3; ++a) {
+        for (const Range& in : ins)
+            if (overlaps(outs[a], in)) return WAN_ATTN_ERR_INVALID_ARG;
+        for (size_t c = a + 1; c < 3; ++c)
+            if (overlaps(outs[a], outs[c])) return WAN_ATTN_ERR_INVALID_ARG;
+    }
+    CUtensorMap tq, tk, tv;
+    if (!make_bshd_map(&tq, q, B, Sq, H, D, 128) || !make_bshd_map(&tk, k, B, Skv, H, D, 64) ||
+        !make_bshd_map(&tv, v, B, Skv, H, D, 64))
+        return WAN_ATTN_ERR_CUDA;
+    FwdParams p{};
+    p.o = o;
+    p.lse = lse;
+    p.B = B;
+    p.S = Sq;
+    p.Skv = Skv;
+    p.H = H;
+    p.mask = mask;
+    p.kv_list = static_cast<const int*>(workspace);
+    p.kv_count = reinterpret_cast<const int*>(static_cast<char*>(workspace) +
+                                              align256(size_t(B) * H * nctas * nkb * 4));
+    p.nqb = nqb;
+    p.nkb = nkb;
+    p.nctas = nctas;
+    p.scale_log2 = static_cast<float>((1.0 / std::sqrt(double(D))) * 1.4426950408889634);
+    p.wait_budget_ns = wait_budget_ns();
+    p.status = device_status_word();
+    if (!p.status) return WAN_ATTN_ERR_CUDA;
+    return launch_fwd_block_sparse(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                       : WAN_ATTN_ERR_CUDA;
 }
 
 // Backward workspace: fp32 dQ accumulator [B, Sq, H, D], fp32 D_i [B, H, Sq] and, for the
@@ -310,6 +367,16 @@ int wan_attn_cross_fwd(const void* q, const void* k, const void* v, void* o, flo
 }
 
 size_t wan_attn_bwd_workspace_size(int B, int S, int H, int D) { return bwd_ws_size(B, S, S, H, D, false); }
+
+size_t wan_attn_fwd_block_sparse_workspace_size(int B, int Sq, int Skv, int H, int D) {
+    return sparse_ws_size(B, Sq, Skv, H, D);
+}
+
+int wan_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const uint8_t* block_mask, int B, int Sq, int Skv, int H, int D, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    return fwd_block_sparse_impl(q, k, v, o, lse, block_mask, B, Sq, Skv, H, D, workspace, workspace_bytes, stream);
+}
 
 int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, int B, int S, int H, int D, void* workspace,

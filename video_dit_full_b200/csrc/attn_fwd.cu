@@ -20,6 +20,14 @@
 //               written back to TMEM as bf16; epilogue O / l -> bf16, LSE.
 // The two Q tiles ping-pong: while one softmax group works on its S, the
 // tensor core runs the other tile's P V and Q K^T.
+//
+// Block-sparse form (template SPARSE): a 64 x 64 block mask selects, for each
+// 64-token query block, the 64-token key blocks it attends (the FastWan / VSA
+// article on the first page: 64 x 64 block-sparse masks).  A CTA walks only
+// the key blocks that any of its 4 query blocks attends, two blocks per K/V
+// stage (each TMA-loaded into one 64-row half, wherever it lies); the softmax
+// sets each row's disallowed halves to -inf.  A row that attends nothing gets
+// O = 0 and LSE = -inf.
 #include <cuda.h>
 
 #include "sm100_ptx.cuh"
@@ -71,6 +79,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
     }
 }
 
+template <bool SPARSE>
 __global__ void __launch_bounds__(NTHREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                 const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
@@ -84,7 +93,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
     const int h = blockIdx.y, b = blockIdx.z;
     const int q0 = blockIdx.x * (NQ * BM);
     const int nq = (q0 + BM < p.S) ? 2 : 1;          // second tile empty on a short tail
-    const int nkv = (p.Skv + BN - 1) / BN;
+    // sparse: this CTA's key blocks, two per K/V step
+    const int* kv_list = nullptr;
+    int kv_count = 0;
+    if constexpr (SPARSE) {
+        const size_t li = (static_cast<size_t>(b) * p.H + h) * p.nctas + blockIdx.x;
+        kv_list = p.kv_list + li * p.nkb;
+        kv_count = p.kv_count[li];
+    }
+    const int nkv = SPARSE ? (kv_count + 1) / 2 : (p.Skv + BN - 1) / BN;
 
     const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sV = base + OFF_V;
     const uint32_t bar0 = base + OFF_BAR;
@@ -118,7 +135,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 
     if (warp == 8) {
         // ------------------------------ TMA producer ------------------------------
-        if (lane == 0) {
+        if (lane == 0 && nkv > 0) {
             tma_prefetch_desc(&tmq);
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
@@ -136,14 +153,34 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 ok = wait_thread(bar(K_EMPTY + s), use ^ 1, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar(K_FULL + s), TILE_BYTES);
-                tma_load_4d_hint(sK + s * TILE_BYTES, &tmk, bar(K_FULL + s), 0, h, j * BN, b, keep);
-                tma_load_4d_hint(sK + s * TILE_BYTES + HALF_BYTES, &tmk, bar(K_FULL + s), 64, h, j * BN, b, keep);
+                if constexpr (SPARSE) {
+                    // two 64-key blocks into rows 0-63 and 64-127 of both 64-wide halves of d (a missing
+                    // second block repeats the first; the softmax masks it)
+                    const int ka = kv_list[2 * j] * 64, kb = kv_list[min(2 * j + 1, kv_count - 1)] * 64;
+                    for (int e = 0; e < 2; ++e) {
+                        const uint32_t dst = sK + s * TILE_BYTES + e * HALF_BYTES;
+                        tma_load_4d_hint(dst, &tmk, bar(K_FULL + s), 64 * e, h, ka, b, keep);
+                        tma_load_4d_hint(dst + HALF_BYTES / 2, &tmk, bar(K_FULL + s), 64 * e, h, kb, b, keep);
+                    }
+                } else {
+                    tma_load_4d_hint(sK + s * TILE_BYTES, &tmk, bar(K_FULL + s), 0, h, j * BN, b, keep);
+                    tma_load_4d_hint(sK + s * TILE_BYTES + HALF_BYTES, &tmk, bar(K_FULL + s), 64, h, j * BN, b, keep);
+                }
                 kpar[s] = use;
                 ok = wait_thread(bar(V_EMPTY + s), use ^ 1, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar(V_FULL + s), TILE_BYTES);
-                tma_load_4d_hint(sV + s * TILE_BYTES, &tmv, bar(V_FULL + s), 0, h, j * BN, b, keep);
-                tma_load_4d_hint(sV + s * TILE_BYTES + HALF_BYTES, &tmv, bar(V_FULL + s), 64, h, j * BN, b, keep);
+                if constexpr (SPARSE) {
+                    const int ka = kv_list[2 * j] * 64, kb = kv_list[min(2 * j + 1, kv_count - 1)] * 64;
+                    for (int e = 0; e < 2; ++e) {
+                        const uint32_t dst = sV + s * TILE_BYTES + e * HALF_BYTES;
+                        tma_load_4d_hint(dst, &tmv, bar(V_FULL + s), 64 * e, h, ka, b, keep);
+                        tma_load_4d_hint(dst + HALF_BYTES / 2, &tmv, bar(V_FULL + s), 64 * e, h, kb, b, keep);
+                    }
+                } else {
+                    tma_load_4d_hint(sV + s * TILE_BYTES, &tmv, bar(V_FULL + s), 0, h, j * BN, b, keep);
+                    tma_load_4d_hint(sV + s * TILE_BYTES + HALF_BYTES, &tmv, bar(V_FULL + s), 64, h, j * BN, b, keep);
+                }
                 vpar[s] = use;
             }
             if (!ok) {
@@ -160,7 +197,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         if (lane == 0) {
             const uint32_t idesc_qk = make_idesc(1, 1, 1, 0, 0, BM, BN);
             const uint32_t idesc_pv = make_idesc(1, 1, 1, 0, 1, BM, HD);
-            bool ok = true;
+            bool ok = nkv > 0;                           // sparse: a CTA may attend no key block
             for (int t = 0; t < nq && ok; ++t) ok = wait_thread(bar(Q_FULL + t), 0, wc);
             if (ok) ok = wait_thread(bar(K_FULL + 0), 0, wc);
             if (ok) {
@@ -219,11 +256,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q * 32]));
             tmem_wait_ld();
             float* s = reinterpret_cast<float*>(sr);
-            const int valid = p.Skv - j * BN;    // keys of this tile that exist
-            if (valid < BN) {
+            if constexpr (SPARSE) {
+                // the two key blocks of this step: each half keeps its keys if the row's query block
+                // attends the block (and the keys exist); a missing second block is masked
+                const int kba = kv_list[2 * j], kbb = (2 * j + 1 < kv_count) ? kv_list[2 * j + 1] : -1;
+                const int qb = min(row, p.S - 1) / 64;
+                const uint8_t* mrow = p.mask + ((static_cast<size_t>(b) * p.H + h) * p.nqb + qb) * p.nkb;
+                const int lim0 = mrow[kba] ? min(64, p.Skv - 64 * kba) : 0;
+                const int lim1 = (kbb >= 0 && mrow[kbb]) ? min(64, p.Skv - 64 * kbb) : 0;
 #pragma unroll
-                for (int q = 0; q < 128; ++q)
-                    if (q >= valid) s[q] = -INFINITY;
+                for (int q = 0; q < 64; ++q) {
+                    if (q >= lim0) s[q] = -INFINITY;
+                    if (q >= lim1) s[64 + q] = -INFINITY;
+                }
+            } else {
+                const int valid = p.Skv - j * BN;    // keys of this tile that exist
+                if (valid < BN) {
+#pragma unroll
+                    for (int q = 0; q < 128; ++q)
+                        if (q >= valid) s[q] = -INFINITY;
+                }
             }
             float mx = s[0];
 #pragma unroll
@@ -236,7 +288,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 m_ref = m_cand;
                 moved = true;
             }
-            const float neg = -m_ref;
+            // sparse: until a row meets its first allowed key, m_ref is -inf and every s is -inf;
+            // subtracting 0 then keeps exp2(-inf) = 0 instead of exp2(-inf + inf)
+            const float neg = (SPARSE && m_ref == -INFINITY) ? 0.f : -m_ref;
             float sum = 0.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -266,10 +320,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             tc_fence_before();
             mbar_arrive(bar(P_FULL + t));
         }
-        if (ok) ok = wait_warp(bar(O_FINAL + t), 0, wc);
+        if (ok && nkv > 0) ok = wait_warp(bar(O_FINAL + t), 0, wc);
         if (ok) {
             tc_fence_after();
-            const float inv_l = 1.f / l;
+            // sparse: a row with no allowed key (l = 0, or no key block at all) gets O = 0, LSE = -inf
+            const bool empty = SPARSE && !(l > 0.f);
+            const float inv_l = empty ? 0.f : 1.f / l;
             __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
                                   ((static_cast<size_t>(b) * p.S + row) * p.H + h) * HD;
 #pragma unroll 1
@@ -282,6 +338,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     pw[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                if (empty) {                                   // TMEM O may never have been written
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pw[e] = 0u;
+                }
                 if (row < p.S) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
@@ -289,7 +349,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 }
             }
             if (row < p.S)
-                p.lse[(static_cast<size_t>(b) * p.H + h) * p.S + row] = (m_ref + log2f(l)) * 0.69314718055994531f;
+                p.lse[(static_cast<size_t>(b) * p.H + h) * p.S + row] =
+                    empty ? -INFINITY : (m_ref + log2f(l)) * 0.69314718055994531f;
         }
     }
 
@@ -303,9 +364,53 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                cudaStream_t stream) {
-    if (configure_smem(reinterpret_cast<const void*>(fwd::attn_fwd_kernel), fwd::SMEM_BYTES) != 0) return -1;
+    if (configure_smem(reinterpret_cast<const void*>(fwd::attn_fwd_kernel<false>), fwd::SMEM_BYTES) != 0) return -1;
     const dim3 grid((p.S + fwd::NQ * fwd::BM - 1) / (fwd::NQ * fwd::BM), p.H, p.B);
-    fwd::attn_fwd_kernel<<<grid, fwd::NTHREADS, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    fwd::attn_fwd_kernel<false><<<grid, fwd::NTHREADS, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+namespace fwd {
+// One warp per (b, h, CTA): the ascending key blocks that any of the CTA's 4 query blocks attends
+// (a ballot over 32 key blocks at a time).
+__global__ void __launch_bounds__(256) sparse_lists_kernel(const uint8_t* __restrict__ mask, int* __restrict__ list,
+                                                           int* __restrict__ count, long long nlists, int nctas,
+                                                           int nqb, int nkb) {
+    const int lane = threadIdx.x & 31;
+    const long long warp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    for (long long w = warp; w < nlists; w += nwarps) {          // w = (b * H + h) * nctas + cta
+        const long long bh = w / nctas;
+        const int cta = static_cast<int>(w - bh * nctas);
+        const int qb0 = cta * 4, nrows = min(4, nqb - qb0);
+        const uint8_t* m = mask + (bh * nqb + qb0) * nkb;
+        int* out = list + w * nkb;
+        int n = 0;
+        for (int k0 = 0; k0 < nkb; k0 += 32) {
+            const int kb = k0 + lane;
+            bool any = false;
+            if (kb < nkb)
+                for (int r = 0; r < nrows; ++r) any |= m[static_cast<long long>(r) * nkb + kb] != 0;
+            const unsigned bal = __ballot_sync(0xffffffffu, any);
+            if (any) out[n + __popc(bal & ((1u << lane) - 1u))] = kb;
+            n += __popc(bal);
+        }
+        if (lane == 0) count[w] = n;
+    }
+}
+}  // namespace fwd
+
+int launch_fwd_block_sparse(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64,
+                            const FwdParams& p, cudaStream_t stream) {
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long nlists = static_cast<long long>(p.B) * p.H * p.nctas;
+    fwd::sparse_lists_kernel<<<sms * 8, 256, 0, stream>>>(p.mask, const_cast<int*>(p.kv_list),
+                                                          const_cast<int*>(p.kv_count), nlists, p.nctas, p.nqb, p.nkb);
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    if (configure_smem(reinterpret_cast<const void*>(fwd::attn_fwd_kernel<true>), fwd::SMEM_BYTES) != 0) return -1;
+    const dim3 grid(p.nctas, p.H, p.B);
+    fwd::attn_fwd_kernel<true><<<grid, fwd::NTHREADS, fwd::SMEM_BYTES, stream>>>(tq, tk64, tv64, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

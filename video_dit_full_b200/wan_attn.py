@@ -29,6 +29,8 @@ SIGNATURES = [
     ("wan_attn_cp_merge", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     ("wan_attn_cp_accumulate", _I, [_P, _P, _P, _Z, _I, _P]),
     ("wan_attn_cp_layout", _I, [_P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    ("wan_attn_fwd_block_sparse_workspace_size", _Z, [_I, _I, _I, _I, _I]),
+    ("wan_attn_fwd_block_sparse", _I, [_P, _P, _P, _P, _F, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
     ("wan_fp8_quantize_rows", _I, [_P, _P, _P, _I, _I, _P]),
     ("wan_fp8_quantize_tensor", _I, [_P, _P, _P, _I, _I, _P]),
     ("wan_fp8_gemm", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
@@ -163,6 +165,34 @@ def cross_fwd(q, k, v, o=None, lse=None, stream=None):
         raise ValueError("lse must be a contiguous fp32 [B, H, Sq] tensor")
     _check("wan_attn_cross_fwd", lib().wan_attn_cross_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                                           lse.data_ptr(), B, Sq, Skv, H, D, _stream_ptr(stream)))
+    return o, lse
+
+
+def block_sparse_workspace_size(B, Sq, Skv, H, D=128) -> int:
+    return lib().wan_attn_fwd_block_sparse_workspace_size(B, Sq, Skv, H, D)
+
+
+def fwd_block_sparse(q, k, v, block_mask, o=None, lse=None, workspace=None, stream=None):
+    """O, LSE of q attending, per 64-token query block, only the 64-token key blocks that
+    block_mask (uint8 [B, H, ceil(Sq/64), ceil(Skv/64)]) allows (``wan_attn_fwd_block_sparse``)."""
+    import torch
+    _check_bshd("q", q)
+    B, Sq, H, D = q.shape
+    Skv = _check_kv(q, k, v)
+    nqb, nkb = (Sq + 63) // 64, (Skv + 63) // 64
+    _check_plain("block_mask", block_mask, torch.uint8, B * H * nqb * nkb)
+    o = torch.empty_like(q) if o is None else o
+    _check_bshd("o", o, q.shape)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Sq) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, Sq] tensor")
+    if workspace is None:
+        workspace = torch.empty(block_sparse_workspace_size(B, Sq, Skv, H, D), dtype=torch.uint8, device=q.device)
+    _check("wan_attn_fwd_block_sparse",
+           lib().wan_attn_fwd_block_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                           block_mask.data_ptr(), B, Sq, Skv, H, D, workspace.data_ptr(),
+                                           workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
     return o, lse
 
 
