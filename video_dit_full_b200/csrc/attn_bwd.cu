@@ -16,8 +16,9 @@
 //                 dV += P^T dO_i                            (A = P^T in TMEM)
 //                 dS^T = P^T (dP^T - D_i)  -> TMEM and smem (into dO_i's buffer)
 //                 dK += dS^T Q_i                            (A = dS^T in TMEM)
-//                 dQ_i^T = K^T dS^T  -> TMEM -> shared (fp32) -> TMA reduce-add into
-//                                       the accumulator (a dedicated reducer warp)
+//                 dQ_i^T = K^T dS^T  -> TMEM (dP^T's columns, so the next tile's S^T can
+//                                       start at once) -> shared (fp32) -> TMA reduce-add
+//                                       into the accumulator (a dedicated reducer warp)
 //               P is recomputed from the forward's LSE; nothing of size S x S is stored.
 //   bwd_dq      dQ = bf16(accumulator / sqrt(D)).
 //
@@ -208,17 +209,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             const uint32_t id_tb = make_idesc(1, 1, 1, 0, 1, BM, HD);   // A in TMEM, B MN-major
             const uint32_t id_mm = make_idesc(1, 1, 1, 1, 1, HD, BM);   // both MN-major
             bool ok = wait_thread(bar(KV_FULL), 0, wc);
+            if (ok) ok = wait_thread(bar(QDO_FULL + 0), 0, wc);
+            if (ok) {
+                tc_fence_after();
+                mma_kmajor(tmem + T_S, sK, sQ(0), id_kk, false);      // S^T = K Q^T of the first tile
+                mma_commit(bar(S_FULL));
+                mma_kmajor(tmem + T_DP, sV, sDO(0), id_kk, false);    // dP^T = V dO^T
+                mma_commit(bar(DP_FULL));
+            }
             for (int i = 0; i < nq && ok; ++i) {
                 const int s = i & 1;
-                ok = wait_thread(bar(QDO_FULL + s), (i >> 1) & 1, wc);
-                if (ok && i > 0) ok = wait_thread(bar(DQ_DRAINED), (i - 1) & 1, wc);
-                if (!ok) break;
-                tc_fence_after();
                 const uint32_t q_s = sQ(s), do_s = sDO(s);
-                mma_kmajor(tmem + T_S, sK, q_s, id_kk, false);        // S^T = K Q^T
-                mma_commit(bar(S_FULL));
-                mma_kmajor(tmem + T_DP, sV, do_s, id_kk, false);      // dP^T = V dO^T
-                mma_commit(bar(DP_FULL));
                 ok = wait_thread(bar(P_READY), i & 1, wc);
                 if (!ok) break;
                 tc_fence_after();
@@ -230,9 +231,26 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 mma_ts_bmn(tmem + T_DK, tmem + T_DP, q_s, id_tb, i > 0);   // dK += dS^T Q
                 ok = wait_thread(bar(DS_SMEM), i & 1, wc);
                 if (!ok) break;
-                mma_ss_mn(tmem + T_S, sK, do_s, id_mm);                    // dQ^T = K^T dS^T (dS^T in dO's buffer)
+                // dQ^T = K^T dS^T (dS^T in dO's buffer) into dP^T's columns, which the dK MMA just
+                // read: S^T's columns are free for the next tile at once
+                mma_ss_mn(tmem + T_DP, sK, do_s, id_mm);
                 mma_commit(bar(DQ_FULL));
                 mma_commit(bar(QDO_EMPTY + s));
+                if (i + 1 < nq) {
+                    // the next tile's S^T runs while the gradient warps copy dQ^T out; its dP^T
+                    // (needed only after its P) once that copy has freed the columns
+                    const int s1 = (i + 1) & 1;
+                    ok = wait_thread(bar(QDO_FULL + s1), ((i + 1) >> 1) & 1, wc);
+                    if (!ok) break;
+                    tc_fence_after();
+                    mma_kmajor(tmem + T_S, sK, sQ(s1), id_kk, false);
+                    mma_commit(bar(S_FULL));
+                    ok = wait_thread(bar(DQ_DRAINED), i & 1, wc);
+                    if (!ok) break;
+                    tc_fence_after();
+                    mma_kmajor(tmem + T_DP, sV, sDO(s1), id_kk, false);
+                    mma_commit(bar(DP_FULL));
+                }
             }
             if (ok) mma_commit(bar(FINAL));
             mma_commit(bar(DRAIN));
@@ -364,7 +382,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll 1
             for (int q = 0; q < 2; ++q) {
                 uint32_t v[32];
-                tmem_ld32(tS + q * 32, v);
+                tmem_ld32(tDP + q * 32, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) stage[(cb + q * 32 + e) * HD + j] = __uint_as_float(v[e]);
