@@ -302,16 +302,27 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         float* s_lse = reinterpret_cast<float*>(smem + OFF_VEC + warp * VEC_BYTES);
         float* s_del = s_lse + 64;
         bool ok = true;
+        // a tile's lse / D come from global memory one tile ahead, so their latency hides
+        // behind the previous tile instead of delaying the wait for S^T
+        float nl[2], nd[2];
+        auto load_vec = [&](int ti) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int qi = (i_first + ti) * BM + cb + e * 32 + lane;
+                nl[e] = qi < Sq ? p.lse[bh * Sq + qi] * LOG2E : INFINITY;
+                nd[e] = qi < Sq ? p.delta[bh * Sq + qi] : 0.f;
+            }
+        };
+        if (nq > 0) load_vec(0);
         for (int i = 0; i < nq && ok; ++i) {
             __syncwarp();                                    // previous tile's values no longer read
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const int col = e * 32 + lane;
-                const int qi = (i_first + i) * BM + cb + col;
-                s_lse[col] = qi < Sq ? p.lse[bh * Sq + qi] * LOG2E : INFINITY;
-                s_del[col] = qi < Sq ? p.delta[bh * Sq + qi] : 0.f;
+                s_lse[e * 32 + lane] = nl[e];
+                s_del[e * 32 + lane] = nd[e];
             }
             __syncwarp();
+            if (i + 1 < nq) load_vec(i + 1);
 
             ok = wait_warp(bar(S_FULL), i & 1, wc);
             if (!ok) break;
