@@ -132,3 +132,36 @@ def test_cross_host_side_validation_without_gpu(built):
     assert lib.wan_attn_cross_bwd(*args(D=256)) == UNSUPPORTED
     assert lib.wan_attn_cross_bwd(*args(dk=v)) == INVALID                 # output aliases an input
     assert lib.wan_attn_cross_bwd(*args(dv=ctypes.c_void_p(dk.value + 64))) == INVALID   # outputs overlap
+
+
+def test_sparse_fp8_cp_host_side_validation_without_gpu(built):
+    from video_dit_full_b200 import wan_attn
+    lib = wan_attn.lib()
+    INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 5
+    P = [ctypes.c_void_p(0x100000 + i * 0x10000000) for i in range(8)]
+    q, k, v, o, lse, mask, ws, z = P
+    # block-sparse: lists int32 [B, H, ceil(Sq/256), ceil(Skv/64)] + lengths, each 256-byte aligned
+    need = lib.wan_attn_fwd_block_sparse_workspace_size(1, 300, 700, 2, 128)
+    a = lambda x: (x + 255) // 256 * 256
+    assert need == a(2 * 2 * 11 * 4) + a(2 * 2 * 4)
+    assert lib.wan_attn_fwd_block_sparse_workspace_size(1, 300, 700, 2, 96) == 0
+    args = [q, k, v, o, lse, mask, 1, 300, 700, 2, 128, ws, need, None]
+    assert lib.wan_attn_fwd_block_sparse(*args[:5], None, *args[6:]) == INVALID          # no mask
+    assert lib.wan_attn_fwd_block_sparse(*args[:10], 64, *args[11:]) == UNSUPPORTED
+    assert lib.wan_attn_fwd_block_sparse(*args[:12], need - 4, None) == WORKSPACE
+    assert lib.wan_attn_fwd_block_sparse(*args[:11], None, need, None) == WORKSPACE
+    assert lib.wan_attn_fwd_block_sparse(q, k, v, q, *args[4:]) == INVALID               # o aliases q
+    # FP8: K a multiple of 16, N of 8, outputs overlap no input
+    assert lib.wan_fp8_quantize_rows(q, k, v, 10, 24, None) == INVALID
+    assert lib.wan_fp8_quantize_rows(q, q, v, 10, 32, None) == INVALID
+    assert lib.wan_fp8_quantize_tensor(q, k, ctypes.c_void_p(v.value + 4), 8, 32, None) == INVALID  # scale2 8-aligned
+    assert lib.wan_fp8_gemm(q, k, v, o, lse, 100, 20, 32, None) == INVALID               # N % 8
+    assert lib.wan_fp8_gemm(q, k, v, o, q, 100, 24, 32, None) == INVALID                 # y aliases the codes
+    assert lib.wan_fp8_gemm(None, k, v, o, lse, 100, 24, 32, None) == INVALID
+    # context parallelism
+    assert lib.wan_attn_cp_accumulate(q, k, None, 12, 1, None) == INVALID                # n % 8
+    assert lib.wan_attn_cp_accumulate(q, ctypes.c_void_p(q.value + 16), None, 64, 0, None) == INVALID
+    assert lib.wan_attn_cp_layout(q, k, 1, 5, 2, 2, 128, 4, None) == INVALID             # no such order
+    assert lib.wan_attn_cp_layout(q, k, 1, 5, 2, 2, 64, 0, None) == UNSUPPORTED
+    assert lib.wan_attn_cp_merge(q, k, q, o, None, 1, 10, 2, 128, 0, None) == INVALID    # o_part aliases o_acc
+    assert lib.wan_attn_cp_merge(q, k, v, None, None, 1, 10, 2, 128, 0, None) == INVALID  # no lse_part

@@ -311,7 +311,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant
 // Barriers: FULL (leader's, counting both CTAs' TMA bytes), EMPTY and TFULL (in each CTA,
 // signalled by the leader's commits), TEMPTY (leader's, 128 arrivals from each CTA).
 // ------------------------------------------------------------------------------------
-constexpr int STAGES2 = 6;
+#ifndef FP8_PAIR_STAGES
+#define FP8_PAIR_STAGES 6
+#endif
+constexpr int STAGES2 = FP8_PAIR_STAGES;            // 32 KB each
 constexpr int HALF_BYTES = 128 * BK, STAGE2_BYTES = 2 * HALF_BYTES;    // A rows | B half rows
 constexpr int OFF_BAR2 = STAGES2 * STAGE2_BYTES;
 enum Bar2 { F2 = 0, E2 = STAGES2, TF2 = 2 * STAGES2, TE2 = 2 * STAGES2 + 2, DR2 = 2 * STAGES2 + 4,
