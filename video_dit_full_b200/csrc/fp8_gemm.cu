@@ -321,7 +321,9 @@ enum Bar2 { F2 = 0, E2 = STAGES2, TF2 = 2 * STAGES2, TE2 = 2 * STAGES2 + 2, DR2 
             NBARS2 = 2 * STAGES2 + 5 };
 constexpr int OFF_TMEM_SLOT2 = OFF_BAR2 + NBARS2 * 8;
 constexpr int OFF_ABORT2 = OFF_TMEM_SLOT2 + 8;
-constexpr int SMEM2_BYTES = OFF_ABORT2 + 8 + 1024;
+constexpr int OFF_EPI2 = (OFF_ABORT2 + 8 + 15) & ~15;   // per epilogue warp: 32 rows x 64 B
+constexpr int EPI_WARP_BYTES = 32 * 64;
+constexpr int SMEM2_BYTES = OFF_EPI2 + 4 * EPI_WARP_BYTES + 1024;
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -491,26 +493,37 @@ fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_con
             if (!ok) break;
             tc_fence_after();
             const int m = m0 + r;
-            const bool row_ok = m < p.M;
-            const float sc = row_ok ? p.a_scales[m] * sw : 0.f;
-            __nv_bfloat16* yrow = reinterpret_cast<__nv_bfloat16*>(p.y) + static_cast<long long>(m) * p.N;
+            const float sc = m < p.M ? p.a_scales[m] * sw : 0.f;
+            // each 32-column chunk goes through the warp's 2 KB of shared memory (row-major,
+            // 16-byte pieces swizzled by row / 2) so that every store writes 8 whole 64-byte
+            // row segments instead of 32 scattered 16-byte pieces
+            uint8_t* wbuf = smem + OFF_EPI2 + (warp - 2) * EPI_WARP_BYTES;
+            const int row0 = m0 + (warp & 3) * 32;                 // this warp's 32 rows
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tmem + b * BN + lane_off + c * 32, v);
                 tmem_wait_ld();
-                const int n = n0 + c * 32;
-                if (row_ok && n < p.N) {
-                    uint4 pk[4];
-                    uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+                uint32_t pw[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pw[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
-                    uint4* dst = reinterpret_cast<uint4*>(yrow + n);
+                for (int e = 0; e < 16; ++e)
+                    pw[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * sc, __uint_as_float(v[2 * e + 1]) * sc);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        if (n + q * 8 < p.N) dst[q] = pk[q];
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4*>(wbuf + lane * 64 + ((q ^ ((lane >> 1) & 3)) * 16)) =
+                        make_uint4(pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
+                __syncwarp();
+                const int n = n0 + c * 32 + (lane & 3) * 8;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int rr = 8 * k + (lane >> 2);
+                    const uint4 val = *reinterpret_cast<const uint4*>(wbuf + rr * 64 + (((lane & 3) ^ ((rr >> 1) & 3)) * 16));
+                    const int mm = row0 + rr;
+                    if (mm < p.M && n < p.N)
+                        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.y) +
+                                                  static_cast<long long>(mm) * p.N + n) = val;
                 }
+                __syncwarp();
             }
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(b));   // leader's TEMPTY[b]
