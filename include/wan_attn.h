@@ -27,6 +27,9 @@
  *   - Kernels never spin without bound: every wait inside a kernel has a time
  *     budget; when one runs out the kernel records WAN_ATTN_ERR_TIMEOUT in a
  *     device status word and exits.  wan_attn_sync_status() reports it.
+ *     While the status word holds an error, a wait that has lasted 1 ms
+ *     gives up too (healthy waits are far shorter), so that the CTAs of a
+ *     call that timed out do not each spend a whole budget.
  */
 #ifndef WAN_ATTN_H
 #define WAN_ATTN_H

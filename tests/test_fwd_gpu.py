@@ -106,3 +106,19 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert wa.sync_status() == 4                  # WAN_ATTN_ERR_TIMEOUT
     assert wa.sync_status() == 0                  # cleared
     check(inputs_for(1, 200, 1, seed=1))          # the context is still usable
+
+
+def test_long_wait_gives_up_early_once_the_device_reported_a_timeout():
+    # after one timeout (status not yet read), a wait that has lasted 1 ms stops at its next
+    # check instead of spending its whole budget: a 10 s budget ends in well under a second
+    import time
+    import torch
+    import video_dit_full_b200 as wa
+    wa.selftest_wait_timeout(2_000_000)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    wa.selftest_wait_timeout(10_000_000_000)
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 1.0
+    assert wa.sync_status() == 4                  # the first timeout, still the one reported
+    assert wa.sync_status() == 0

@@ -7,10 +7,11 @@
   (the workload's bar).  The recipe's own error on N(0,1) inputs is ~3.9e-2
   (the fp64 simulation ``oracle.quant8.attn_fwd_q8_sim``), so the kernel must
   add almost nothing.  The distance to that simulation is reported; it is a
-  gate (<= 5e-3) only when every key fits one 128-key tile, since the kernel
-  quantises P against the running maximum and the simulation against the
-  final one (the same value once a single tile holds all keys).
-* Exact cases: Q = 0 gives O = the mean of the dequantised V.
+  gate (<= 5e-3) only when every key fits the kernel's first 64-key step,
+  since the kernel quantises P against the running maximum and the simulation
+  against the final one (the same value once a single step holds all keys).
+* Exact cases: Q = 0 gives O = the mean of the dequantised V (LSE = ln S to the
+  error bound of the kernel's polynomial exponentials).
 * LSE of the dequantised scores: within 2e-2 of the exact LSE (int8 score
   error ~1.4e-2 per score, averaged by the log-sum-exp).
 """
@@ -66,7 +67,7 @@ def check(x, rows=None):
     print(f"q8 O rel-frob vs exact {rel:.3e} (recipe alone {rel_recipe:.3e}, kernel vs recipe {rel_sim:.3e}) "
           f"max-abs {max_abs:.3e} LSE {lse_err:.3e}")
     assert rel <= REL_FROB, rel
-    if x["q"].shape[1] <= 128:
+    if x["q"].shape[1] <= 64:
         assert rel_sim <= 5e-3, rel_sim
     assert lse_err <= 2e-2, lse_err
 
@@ -97,4 +98,7 @@ def test_q8_uniform_scores_give_mean_of_dequantised_v():
     got = bf16_to_f64(o)
     _, rel = errors(got, np.broadcast_to(want, got.shape))
     assert rel <= 4e-3, rel                      # bf16 output rounding only
-    np.testing.assert_allclose(lse.cpu().numpy(), np.log(S), atol=1e-5)
+    # LSE = ln l; part of the kernel's exponentials come from a degree-2 polynomial with relative
+    # error <= 1.73e-3 (far below e4m3's half step 2^-4, which P is rounded to), so l is exact
+    # to that factor and LSE to ln(1 + 1.73e-3) < 2e-3
+    np.testing.assert_allclose(lse.cpu().numpy(), np.log(S), atol=2e-3)

@@ -61,14 +61,14 @@ bool make_bshd_map(CUtensorMap* m, const void* base, int B, int S, int H, int D,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tensor map over an 8-bit [B*H, S, 128] tensor viewed as 3-D (128, S, B*H), box (128, 128, 1),
+// Tensor map over an 8-bit [B*H, S, 128] tensor viewed as 3-D (128, S, B*H), box (128, rows, 1),
 // 128-byte swizzle (one 128-byte row per token), tokens past S read as zero.
-bool make_bh_s_d8_map(CUtensorMap* m, const void* base, int BH, int S) {
+bool make_bh_s_d8_map(CUtensorMap* m, const void* base, int BH, int S, int rows) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     const cuuint64_t dims[3] = {128, (cuuint64_t)S, (cuuint64_t)BH};
     const cuuint64_t strides[2] = {128, (cuuint64_t)S * 128};
-    const cuuint32_t box[3] = {128, 128, 1};
+    const cuuint32_t box[3] = {128, (cuuint32_t)rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -438,8 +438,8 @@ int wan_attn_fwd_q8(const void* q, const void* k, const void* v, void* o, float*
     qp.H = H;
     qp.nblk = nblk;
     CUtensorMap tq, tk, tv;
-    if (!make_bh_s_d8_map(&tq, qp.q8, B * H, S) || !make_bh_s_d8_map(&tk, qp.k8, B * H, S) ||
-        !make_bh_s_d8_map(&tv, qp.v8, B * H, S))
+    if (!make_bh_s_d8_map(&tq, qp.q8, B * H, S, 128) || !make_bh_s_d8_map(&tk, qp.k8, B * H, S, 64) ||
+        !make_bh_s_d8_map(&tv, qp.v8, B * H, S, 64))
         return WAN_ATTN_ERR_CUDA;
     Q8AttnParams p;
     p.o = o;

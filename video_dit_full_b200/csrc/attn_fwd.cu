@@ -256,18 +256,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q * 32]));
             tmem_wait_ld();
             float* s = reinterpret_cast<float*>(sr);
+            // keys kept in each 64-column half; in the sparse kernel a half its row does not attend
+            // (lim 0) is left out of the max and the exponentials and gets P = 0
+            int lim0 = 64, lim1 = 64;
             if constexpr (SPARSE) {
                 // the two key blocks of this step: each half keeps its keys if the row's query block
-                // attends the block (and the keys exist); a missing second block is masked
+                // attends the block (and the keys exist); a missing second block is masked.  A
+                // warp's 32 rows lie in one 64-row query block, so lim0 and lim1 are warp-uniform.
                 const int kba = kv_list[2 * j], kbb = (2 * j + 1 < kv_count) ? kv_list[2 * j + 1] : -1;
                 const int qb = min(row, p.S - 1) / 64;
                 const uint8_t* mrow = p.mask + ((static_cast<size_t>(b) * p.H + h) * p.nqb + qb) * p.nkb;
-                const int lim0 = mrow[kba] ? min(64, p.Skv - 64 * kba) : 0;
-                const int lim1 = (kbb >= 0 && mrow[kbb]) ? min(64, p.Skv - 64 * kbb) : 0;
+                lim0 = mrow[kba] ? min(64, p.Skv - 64 * kba) : 0;
+                lim1 = (kbb >= 0 && mrow[kbb]) ? min(64, p.Skv - 64 * kbb) : 0;
+                if (lim0 > 0 && lim0 < 64) {                       // a short last key block
 #pragma unroll
-                for (int q = 0; q < 64; ++q) {
-                    if (q >= lim0) s[q] = -INFINITY;
-                    if (q >= lim1) s[64 + q] = -INFINITY;
+                    for (int q = 0; q < 64; ++q)
+                        if (q >= lim0) s[q] = -INFINITY;
+                }
+                if (lim1 > 0 && lim1 < 64) {
+#pragma unroll
+                    for (int q = 0; q < 64; ++q)
+                        if (q >= lim1) s[64 + q] = -INFINITY;
                 }
             } else {
                 const int valid = p.Skv - j * BN;    // keys of this tile that exist
@@ -277,9 +286,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                         if (q >= valid) s[q] = -INFINITY;
                 }
             }
-            float mx = s[0];
+            // row max of each half: 4 chains of three-input maxima
+            auto half_max = [&](int h0) {
+                float m4[4];
 #pragma unroll
-            for (int q = 1; q < 128; ++q) mx = fmaxf(mx, s[q]);
+                for (int q = 0; q < 4; ++q) m4[q] = fmax3(s[h0 + q], s[h0 + q + 4], s[h0 + q + 8]);
+#pragma unroll
+                for (int e = 12; e + 8 <= 64; e += 8)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], s[h0 + e + q], s[h0 + e + 4 + q]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], s[h0 + 60 + q]);
+                return fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+            };
+            float mx = -INFINITY;
+            if (lim0 > 0) mx = half_max(0);
+            if (lim1 > 0) mx = fmaxf(mx, half_max(64));
             const float m_cand = mx * c;
             float alpha = 1.f;
             bool moved = false;
@@ -295,6 +317,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
+                if (SPARSE && (half == 0 ? lim0 : lim1) == 0) {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) pk[q] = 0u;
+                    tmem_st32(tS + half * 32, pk);
+                    continue;
+                }
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const float p0 = ex2_approx(fmaf(s[half * 64 + 2 * q], c, neg));

@@ -15,13 +15,13 @@
 //                 nearest even), written
 //                 head-major [B, H, S, 128] into the workspace.
 //   q8_attn       one CTA per pair of 128-row Q tiles of one (b, h), sharing
-//                 128-key K8/V8 tiles (three-stage TMA rings); the same ping-pong
-//                 as the bf16 forward:
+//                 64-key K8/V8 tiles (six-stage TMA rings), one quantisation block
+//                 per step, S double-buffered in TMEM per Q tile:
 //                   S_t = Q8_t K8^T         kind::i8, int32 in TMEM
 //                   s = S sQ sK / sqrt(D) * log2(e) per 64-key column block
 //                   P8_t = e4m3(2^(s - m + log2(P_SCALE sV_blk / sV_max)))  -> TMEM (over S_t)
 //                   O_t += P8_t V8        kind::f8f6f4, fp32 accumulator in TMEM
-//                 warp 8 TMA, warp 9 MMA, warps 0-3 / 4-7 softmax of Q tile 0 / 1.
+//                 warp 8 TMA, warps 9 / 10 MMA, warps 0-3 / 4-7 softmax of Q tile 0 / 1.
 #include <cuda.h>
 
 #include "sm100_ptx.cuh"
@@ -129,30 +129,48 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const Q8QuantParams p)
 }
 
 constexpr int BM = 128;                     // query rows per Q tile
-constexpr int BN = 128;                     // keys per K/V tile (two quantisation blocks)
+constexpr int BN = 64;                      // keys per step: one quantisation block
 constexpr int NQ = 2;                       // Q tiles per CTA (they share every K/V tile)
-constexpr int T8 = BM * HD;                 // 16 KB 8-bit tile
-constexpr int STAGES = 3;
+constexpr int TQ8 = BM * HD;                // 16 KB 8-bit Q tile
+constexpr int TKV8 = BN * HD;               // 8 KB 8-bit K or V tile
+constexpr int STAGES = 6;
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + NQ * T8;
-constexpr int OFF_V = OFF_K + STAGES * T8;
-constexpr int OFF_RED = OFF_V + STAGES * T8;          // 16 floats: per-warp partial maxima of sV
+constexpr int OFF_K = OFF_Q + NQ * TQ8;
+constexpr int OFF_V = OFF_K + STAGES * TKV8;
+constexpr int OFF_RED = OFF_V + STAGES * TKV8;        // 16 floats: per-warp partial maxima of sV
 constexpr int OFF_BAR = OFF_RED + 64;
-enum Bar { Q_FULL = 0, K_FULL = 2, K_EMPTY = 5, V_FULL = 8, V_EMPTY = 11, S_FULL = 14, P_FULL = 16,
-           O_FINAL = 18, DRAIN = 20, NBARS = 21 };
+// KV_FULL + s / KV_EMPTY + s: K and V of one 64-key block, loaded and released together;
+// S_FULL + 2 t + b: S of Q tile t in buffer b is ready; P_FULL + 2 t + b: P of tile t in buffer
+// b is; PV_LAST + t: P V of the next-to-last block has landed in O; O_FINAL + t: the last has.
+// Per-buffer barriers keep each waiter at most one phase behind its barrier: the softmax may
+// finish steps j and j + 1 before the MMA takes P of step j, but not step j + 2 (its S is
+// computed only after that), so a parity names the phase without ambiguity.
+enum Bar { Q_FULL = 0, KV_FULL = 2, KV_EMPTY = KV_FULL + STAGES, S_FULL = KV_EMPTY + STAGES,
+           P_FULL = S_FULL + 4, PV_LAST = P_FULL + 4, O_FINAL = PV_LAST + 2, DRAIN = O_FINAL + 2,
+           NBARS = DRAIN + 2 };
 constexpr int OFF_TMEM_SLOT = OFF_BAR + NBARS * 8;
 constexpr int OFF_ABORT = OFF_TMEM_SLOT + 8;
 constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
-constexpr int NTHREADS = 320;               // warps 0-3 softmax of Q tile 0, 4-7 of Q tile 1, 8 TMA, 9 MMA
-constexpr uint32_t TMEM_COLS = 512;         // S0 | S1 (int32; P8 over their first 32 columns) | O0 | O1
+// warps 0-3 softmax of Q tile 0, 4-7 of Q tile 1, 8 TMA, 9 and 10 the MMAs of Q tile 0 and 1: one
+// issuing thread per tile, so that the two tiles' MMA chains do not queue behind each other
+constexpr int NTHREADS = 352;
+// TMEM: S of tile t, buffer b (int32, 64 columns; P8 over its first 16) at 64 (2 t + b); O of
+// tile t (fp32, 128 columns) at 256 + 128 t.  With S double-buffered, the MMA computes the next
+// S of a tile while its softmax works on this one.
+constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t T_O = 256;
 // The running max is moved only when it rises by more than 1 (log2 units), so p <= 2 against
 // the max in use; P is then quantised as e4m3(P_SCALE * p * sV_block / sV_max) <= 448.
 constexpr float RESCALE_THRESHOLD = 1.0f;
+#ifndef WAN_Q8_POLY_GROUPS
+#define WAN_Q8_POLY_GROUPS 3        // of every 8 groups of 4 exponentials in P, this many use exp2_poly2_x2
+#endif
+constexpr int Q8_POLY_GROUPS = WAN_Q8_POLY_GROUPS;
 constexpr float P_SCALE = 224.f;
 constexpr float LOG2_P_SCALE = 7.807354922057604f;
 
-// S (int32) = Q8 K8^T: both [128 rows][128 bytes] K-major with the 128-byte swizzle, K = 32 per MMA.
+// S (int32) = Q8 K8^T: Q [128 rows][128 bytes], K [64 rows][128 bytes], both K-major with the
+// 128-byte swizzle, K = 32 per MMA.
 __device__ __forceinline__ void issue_qk8(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem, uint32_t idesc) {
 #pragma unroll
     for (int kk = 0; kk < HD / 32; ++kk)
@@ -160,9 +178,10 @@ __device__ __forceinline__ void issue_qk8(uint32_t d_tmem, uint32_t q_smem, uint
                   idesc, kk > 0 ? 1u : 0u);
 }
 
-// O (fp32, TMEM) += P8 V8: P8 in TMEM (4 e4m3 per column, columns 0-31), V8 [key][d] MN-major
-// (one 128-byte swizzle atom spans all 128 d), 32 keys per MMA.  The tensor core's fp32
-// accumulator carries the sum across every 64-key block; each block's V scale is already in P8.
+// O (fp32, TMEM) += P8 V8: P8 in TMEM (4 e4m3 per column, 16 columns for the 64 keys), V8
+// [key][d] MN-major (one 128-byte swizzle atom spans all 128 d), 32 keys per MMA.  The tensor
+// core's fp32 accumulator carries the sum across every 64-key block; each block's V scale is
+// already in P8.
 __device__ __forceinline__ void issue_pv8(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc,
                                           bool accumulate) {
 #pragma unroll
@@ -186,7 +205,7 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
     const int q0 = blockIdx.x * (NQ * BM);
     const int S = p.S;
     const int nq = (q0 + BM < S) ? 2 : 1;
-    const int nkv = (S + BN - 1) / BN;
+    const int nkv = (S + BN - 1) / BN;             // = the number of 64-token blocks
 
     const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sV = base + OFF_V;
     float* red = reinterpret_cast<float*>(smem + OFF_RED);
@@ -205,20 +224,21 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         if (lane == 0) red[warp] = mv;
     }
     if (threadIdx.x == 0) {
-        mbar_init(bar(Q_FULL), 1);
-        mbar_init(bar(Q_FULL + 1), 1);
+        for (int t = 0; t < NQ; ++t) mbar_init(bar(Q_FULL + t), 1);
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(bar(K_FULL + s), 1);
-            mbar_init(bar(K_EMPTY + s), 1);
-            mbar_init(bar(V_FULL + s), 1);
-            mbar_init(bar(V_EMPTY + s), 1);
+            mbar_init(bar(KV_FULL + s), 1);
+            mbar_init(bar(KV_EMPTY + s), nq);         // released by each tile's MMA thread
         }
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(bar(S_FULL + t), 1);
-            mbar_init(bar(P_FULL + t), BM);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar(S_FULL + i), 1);
+            mbar_init(bar(P_FULL + i), BM);
+        }
+        for (int t = 0; t < NQ; ++t) {
+            mbar_init(bar(PV_LAST + t), 1);
             mbar_init(bar(O_FINAL + t), 1);
         }
         mbar_init(bar(DRAIN), 1);
+        mbar_init(bar(DRAIN + 1), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -241,83 +261,73 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
             for (int t = 0; t < nq; ++t) {
-                mbar_arrive_expect_tx(bar(Q_FULL + t), T8);
-                tma_load_3d(sQ + t * T8, &tmq, bar(Q_FULL + t), 0, q0 + t * BM, bh);
+                mbar_arrive_expect_tx(bar(Q_FULL + t), TQ8);
+                tma_load_3d(sQ + t * TQ8, &tmq, bar(Q_FULL + t), 0, q0 + t * BM, bh);
             }
-            int kpar[STAGES], vpar[STAGES];
-            for (int s = 0; s < STAGES; ++s) kpar[s] = vpar[s] = -1;
+            int par[STAGES];
+            for (int s = 0; s < STAGES; ++s) par[s] = -1;
             bool ok = true;
             for (int j = 0; j < nkv; ++j) {
                 const int s = j % STAGES;
                 const int use = (j / STAGES) & 1;
-                ok = wait_thread(bar(K_EMPTY + s), use ^ 1, wc);
+                ok = wait_thread(bar(KV_EMPTY + s), use ^ 1, wc);
                 if (!ok) break;
-                mbar_arrive_expect_tx(bar(K_FULL + s), T8);
-                tma_load_3d(sK + s * T8, &tmk, bar(K_FULL + s), 0, j * BN, bh);
-                kpar[s] = use;
-                ok = wait_thread(bar(V_EMPTY + s), use ^ 1, wc);
-                if (!ok) break;
-                mbar_arrive_expect_tx(bar(V_FULL + s), T8);
-                tma_load_3d(sV + s * T8, &tmv, bar(V_FULL + s), 0, j * BN, bh);
-                vpar[s] = use;
+                mbar_arrive_expect_tx(bar(KV_FULL + s), 2 * TKV8);
+                tma_load_3d(sK + s * TKV8, &tmk, bar(KV_FULL + s), 0, j * BN, bh);
+                tma_load_3d(sV + s * TKV8, &tmv, bar(KV_FULL + s), 0, j * BN, bh);
+                par[s] = use;
             }
             if (!ok) {
                 for (int t = 0; t < nq; ++t) drain_wait(bar(Q_FULL + t), 0);
-                for (int s = 0; s < STAGES; ++s) {
-                    if (kpar[s] >= 0) drain_wait(bar(K_FULL + s), kpar[s]);
-                    if (vpar[s] >= 0) drain_wait(bar(V_FULL + s), vpar[s]);
-                }
+                for (int s = 0; s < STAGES; ++s)
+                    if (par[s] >= 0) drain_wait(bar(KV_FULL + s), par[s]);
             }
         }
-    } else if (warp == 9) {
-        // ------------------------------ MMA issuer --------------------------------
-        if (lane == 0) {
+    } else if (warp >= 9) {
+        // ----------------------- MMA issuer of Q tile t = warp - 9 ------------------------
+        // S(t, j) goes to buffer j % 2.  S of the first two steps is computed up front; after
+        // P(t, j) V(j) the MMA issues S(t, j + 2) into the buffer P(t, j) has just been read
+        // from (the tensor core executes one thread's MMAs in order).
+        const int t = warp - 9;
+        if (lane == 0 && t < nq) {
             const uint32_t idesc_qk = make_idesc(2, 1, 1, 0, 0, BM, BN);   // s32 <- s8 x s8
             const uint32_t idesc_pv = make_idesc(1, 0, 0, 0, 1, BM, HD);   // f32 <- e4m3 x e4m3, V MN-major
-            bool ok = true;
-            for (int t = 0; t < nq && ok; ++t) ok = wait_thread(bar(Q_FULL + t), 0, wc);
-            if (ok) ok = wait_thread(bar(K_FULL + 0), 0, wc);
-            if (ok) {
+            const uint32_t tq = sQ + t * TQ8, to = tmem + T_O + t * HD;
+            auto sbuf = [&](int j) { return tmem + static_cast<uint32_t>((2 * t + (j & 1)) * BN); };
+            bool ok = wait_thread(bar(Q_FULL + t), 0, wc);
+            for (int j = 0; j < 2 && j < nkv && ok; ++j) {
+                ok = wait_thread(bar(KV_FULL + j), 0, wc);
+                if (!ok) break;
                 tc_fence_after();
-                for (int t = 0; t < nq; ++t) {
-                    issue_qk8(tmem + t * BN, sQ + t * T8, sK, idesc_qk);
-                    mma_commit(bar(S_FULL + t));
-                }
-                mma_commit(bar(K_EMPTY + 0));
+                issue_qk8(sbuf(j), tq, sK + j * TKV8, idesc_qk);
+                mma_commit(bar(S_FULL + 2 * t + j));
             }
             for (int j = 0; j < nkv && ok; ++j) {
                 const int s = j % STAGES;
-                const int s1 = (j + 1) % STAGES;
-                ok = wait_thread(bar(V_FULL + s), (j / STAGES) & 1, wc);
-                for (int t = 0; t < nq && ok; ++t) {
-                    ok = wait_thread(bar(P_FULL + t), j & 1, wc);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv8(tmem + T_O + t * HD, tmem + t * BN, sV + s * T8, idesc_pv, j > 0);
-                    if (j + 1 == nkv) mma_commit(bar(O_FINAL + t));
-                    if (j + 1 < nkv) {
-                        if (t == 0) {
-                            ok = wait_thread(bar(K_FULL + s1), ((j + 1) / STAGES) & 1, wc);
-                            if (!ok) break;
-                            tc_fence_after();
-                        }
-                        issue_qk8(tmem + t * BN, sQ + t * T8, sK + s1 * T8, idesc_qk);   // after P V read it
-                        mma_commit(bar(S_FULL + t));
-                    }
-                }
+                const int j2 = j + 2, s2 = j2 % STAGES;
+                const bool next = j2 < nkv;
+                // K and V of block j arrived together (K's wait was two steps ago)
+                if (next) ok = wait_thread(bar(KV_FULL + s2), (j2 / STAGES) & 1, wc);
+                if (ok) ok = wait_thread(bar(P_FULL + 2 * t + (j & 1)), (j >> 1) & 1, wc);
                 if (!ok) break;
-                mma_commit(bar(V_EMPTY + s));
-                if (j + 1 < nkv) mma_commit(bar(K_EMPTY + s1));
+                tc_fence_after();
+                issue_pv8(to, sbuf(j), sV + s * TKV8, idesc_pv, j > 0);
+                mma_commit(bar(KV_EMPTY + s));               // after K(j)'s and V(j)'s last readers
+                if (j + 2 == nkv) mma_commit(bar(PV_LAST + t));
+                if (j + 1 == nkv) mma_commit(bar(O_FINAL + t));
+                if (next) {
+                    issue_qk8(sbuf(j), tq, sK + s2 * TKV8, idesc_qk);
+                    mma_commit(bar(S_FULL + 2 * t + (j & 1)));
+                }
             }
-            mma_commit(bar(DRAIN));
-            drain_wait(bar(DRAIN), 0);
+            mma_commit(bar(DRAIN + t));
+            drain_wait(bar(DRAIN + t), 0);
         }
     } else {
         // ---------------- softmax, O rescale and epilogue (row r of Q tile t) ------------
         const int t = warp >> 2;
         const int r = threadIdx.x & 127;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + t * BN + lane_off;
         const uint32_t tO = tmem + T_O + t * HD + lane_off;
         const int row = q0 + t * BM + r;
         const float* sk = p.sk + static_cast<size_t>(bh) * p.nblk;
@@ -325,88 +335,121 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         const int sv_max_exp = static_cast<int>(__float_as_uint(sv_max) >> 23);   // positive, normal
         float m_ref = -INFINITY, l = 0.f;
         bool ok = (t < nq);
+        // the step's K and V block scales, loaded one step ahead
+        float sk_cur = sk[0], sv_cur = sv[0];
         for (int j = 0; j < nkv && ok; ++j) {
-            ok = wait_warp(bar(S_FULL + t), j & 1, wc);
+            const float sk_next = j + 1 < nkv ? sk[j + 1] : 0.f;
+            const float sv_next = j + 1 < nkv ? sv[j + 1] : 0.f;
+            ok = wait_warp(bar(S_FULL + 2 * t + (j & 1)), (j >> 1) & 1, wc);
             if (!ok) break;
             tc_fence_after();
-            uint32_t sr[128];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[q * 32]));
-            tmem_wait_ld();
-            const int kb = 2 * j;
-            const bool has_b = kb + 1 < p.nblk;
-            const float ca = sq_row * sk[kb] * p.scale_log2;
-            const float cb = has_b ? sq_row * sk[kb + 1] * p.scale_log2 : 0.f;
-            float* s = reinterpret_cast<float*>(sr);
-            // int32 -> fp32 without the conversion unit: |S| <= 128*127*127 < 2^22, so adding
-            // 1.5*2^23 as a float bit pattern and subtracting it back is exact.  Pairs of scores
-            // go through packed fp32 instructions (FADD2 / FMUL2).
-            {
-                const float2 k2 = make_float2(-12582912.f, -12582912.f);
-                const float2 ca2 = make_float2(ca, ca), cb2 = make_float2(cb, cb);
-#pragma unroll
-                for (int c = 0; c < 128; c += 2) {
-                    const float2 xm = make_float2(__int_as_float(static_cast<int>(sr[c]) + 0x4B400000),
-                                                  __int_as_float(static_cast<int>(sr[c + 1]) + 0x4B400000));
-                    const float2 v = fmul2(fadd2(xm, k2), c < 64 ? ca2 : cb2);
-                    s[c] = v.x;
-                    s[c + 1] = v.y;
-                }
-            }
-            const int valid = S - j * BN;
-            if (valid < BN) {
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c >= valid) s[c] = -INFINITY;
-            }
-            // row max: 8 chains of three-input maxima, then a short tree
-            float m8[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) m8[q] = fmax3(s[q], s[q + 8], s[q + 16]);
-#pragma unroll
-            for (int q = 24; q < 128; q += 16)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) m8[e] = (q + 8 + e < 128) ? fmax3(m8[e], s[q + e], s[q + 8 + e])
-                                                                       : fmaxf(m8[e], s[q + e]);
-            m8[0] = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-            float alpha = 1.f;
-            bool moved = false;
-            if (m8[0] > m_ref + RESCALE_THRESHOLD) {
-                alpha = ex2_approx(m_ref - m8[0]);
-                m_ref = m8[0];
-                moved = true;
-            }
+            const uint32_t tS = tmem + static_cast<uint32_t>((2 * t + (j & 1)) * BN) + lane_off;
+            const int valid = S - j * BN;                    // keys of this block that exist
+            // c > 0 even for an all-zero block, so that -inf * c stays -inf below
+            const float c = fmaxf(sq_row * sk_cur * p.scale_log2, 1e-30f);
             // P_SCALE * p * sV_blk / sV_max = 2^(s - m_ref + lg_blk), lg_blk = log2(P_SCALE * sV_blk / sV_max)
             // V block scales are normal powers of two: r = sV_blk / sV_max = 2^-k exactly, k read off
             // the exponent fields
             // (k is clamped to 64: any block 2^-20 below the largest already quantises to zero)
-            const int ka = min(sv_max_exp - static_cast<int>(__float_as_uint(sv[kb]) >> 23), 64);
-            const int kbb = has_b ? min(sv_max_exp - static_cast<int>(__float_as_uint(sv[kb + 1]) >> 23), 64) : 0;
-            const float inv_a = __uint_as_float(static_cast<uint32_t>(127 + ka) << 23) * (1.f / P_SCALE);
-            const float inv_b = __uint_as_float(static_cast<uint32_t>(127 + kbb) << 23) * (1.f / P_SCALE);
-            const float ba = m_ref - (LOG2_P_SCALE - static_cast<float>(ka));
-            const float bbias = m_ref - (LOG2_P_SCALE - static_cast<float>(kbb));
-            float2 sa2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            float2 sb2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            const float2 nba = make_float2(-ba, -ba), nbb = make_float2(-bbias, -bbias);
-            uint32_t pk[32];
+            const int kx = min(sv_max_exp - static_cast<int>(__float_as_uint(sv_cur) >> 23), 64);
+            const float inv = __uint_as_float(static_cast<uint32_t>(127 + kx) << 23) * (1.f / P_SCALE);
+            const float2 c2 = make_float2(c, c);
+            const float2 magic2 = make_float2(12582912.f, 12582912.f);
+            uint32_t pk[16];
+            float sum = 0.f, mx = -INFINITY;
+            // One pass over the row's 64 scores of this block: P8 and the row sum against the
+            // max m, and with `with_max` the block's max.  int32 -> float without the
+            // conversion unit: |S| <= 128*127*127 < 2^22, so the bit pattern of S + 0x4B400000
+            // is the float 1.5*2^23 + S, exactly and in S's order (the max is taken over those
+            // floats); then xm - 1.5*2^23 = S exactly and s - bias = S c - bias in one fused
+            // multiply-add per pair.
+            uint32_t sr[64];
+            float* xm = reinterpret_cast<float*>(sr);
+            auto load = [&]() {
+                tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_wait_ld();
 #pragma unroll
-            for (int w = 0; w < 32; ++w) {
-                const float2 nb = w < 16 ? nba : nbb;
-                const float2 x01 = fadd2(make_float2(s[4 * w], s[4 * w + 1]), nb);
-                const float2 x23 = fadd2(make_float2(s[4 * w + 2], s[4 * w + 3]), nb);
-                const float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
-                const float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-                if (w < 16) sa2[w & 1] = fadd2(sa2[w & 1], fadd2(p01, p23));
-                else sb2[w & 1] = fadd2(sb2[w & 1], fadd2(p01, p23));
-                pk[w] = pack_e4m3x2(p01.x, p01.y) | (pack_e4m3x2(p23.x, p23.y) << 16);
+                for (int e = 0; e < 64; ++e) sr[e] += 0x4B400000u;
+                if (valid < BN) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e)
+                        if (e >= valid) xm[e] = -INFINITY;
+                }
+            };
+            auto pass = [&](float m, bool with_max) {
+                const float nb = -(m - (LOG2_P_SCALE - static_cast<float>(kx)));
+                const float2 n2 = make_float2(nb, nb);
+                float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int w = 0; w < 16; ++w) {
+                    if (with_max)
+                        m4[w & 3] = fmax3(fmax3(m4[w & 3], xm[4 * w], xm[4 * w + 1]), xm[4 * w + 2], xm[4 * w + 3]);
+                    const float2 x01 = ffma2(fsub2(make_float2(xm[4 * w], xm[4 * w + 1]), magic2), c2, n2);
+                    const float2 x23 = ffma2(fsub2(make_float2(xm[4 * w + 2], xm[4 * w + 3]), magic2), c2, n2);
+                    float2 p01, p23;
+                    if ((w & 7) < Q8_POLY_GROUPS) {
+                        p01 = exp2_poly2_x2(x01);
+                        p23 = exp2_poly2_x2(x23);
+                    } else {
+                        p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+                        p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+                    }
+                    sum2[w & 1] = fadd2(sum2[w & 1], fadd2(p01, p23));
+                    pk[w] = pack_e4m3x2(p01.x, p01.y) | (pack_e4m3x2(p23.x, p23.y) << 16);
+                }
+                sum = (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
+                if (with_max) mx = (fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) - 12582912.f) * c;
+            };
+            // P is computed against the max in use while the block's max is found in the same
+            // pass; a row whose max moves is redone against the new max (warp-wide, as TMEM loads
+            // are; after the first few blocks this is rare, and the first block always is).
+#if WAN_Q8_SPECULATE
+            load();
+            pass(m_ref, true);
+#else
+            load();
+            {
+                float m4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) m4[q] = fmax3(xm[q], xm[q + 4], xm[q + 8]);
+#pragma unroll
+                for (int e = 12; e + 8 <= 64; e += 8)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], xm[e + q], xm[e + 4 + q]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], xm[60 + q]);
+                mx = (fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) - 12582912.f) * c;
             }
-            tmem_st32(tS, pk);                                   // P8 over S's first 32 columns
-            // the row sum counts p itself: scale each block's sum by 1 / (P_SCALE * r_blk) = 2^k / P_SCALE
-            const float sum = ((sa2[0].x + sa2[0].y) + (sa2[1].x + sa2[1].y)) * inv_a +
-                              ((sb2[0].x + sb2[0].y) + (sb2[1].x + sb2[1].y)) * inv_b;
-            l = l * alpha + sum;
-            if (j > 0 && __any_sync(0xffffffffu, moved)) {
+#endif
+            float alpha = 1.f;
+            bool moved = false;
+            if (mx > m_ref + RESCALE_THRESHOLD) {
+                alpha = ex2_approx(m_ref - mx);
+                m_ref = mx;
+                moved = true;
+            }
+            const bool any_moved = __any_sync(0xffffffffu, moved);
+#if WAN_Q8_SPECULATE
+            if (any_moved) {
+                load();
+                pass(m_ref, false);
+            }
+#else
+            pass(m_ref, false);
+#endif
+            tmem_st16(tS, pk);                                   // P8 over S's first 16 columns
+            // the row sum counts p itself: scale by 1 / (P_SCALE * r_blk) = 2^k / P_SCALE
+            l = l * alpha + sum * inv;
+            if (j > 0 && any_moved) {
+                // O must hold P(j - 1) V(j - 1) before it is rescaled.  S(t, j + 1) is computed
+                // after that product (the tile's MMAs run in order), so its barrier says so; the
+                // last block, which has no S(t, j + 1), has PV_LAST.
+                ok = (j + 1 < nkv) ? wait_warp(bar(S_FULL + 2 * t + ((j + 1) & 1)), ((j + 1) >> 1) & 1, wc)
+                                   : wait_warp(bar(PV_LAST + t), 0, wc);
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll 1
                 for (int q = 0; q < 4; ++q) {
                     uint32_t o[32];
@@ -419,7 +462,9 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(P_FULL + t));
+            mbar_arrive(bar(P_FULL + 2 * t + (j & 1)));
+            sk_cur = sk_next;
+            sv_cur = sv_next;
         }
         if (ok) ok = wait_warp(bar(O_FINAL + t), 0, wc);
         if (ok) {

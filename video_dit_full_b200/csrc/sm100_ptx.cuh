@@ -63,17 +63,27 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // Control block for bounded waits: a CTA-wide abort flag in shared memory and
 // a time budget.  A wait that runs out of time sets the flag and the device
 // status word; every other wait of the CTA then gives up at its next check.
+// A wait that has already lasted kStatusPollNs (no healthy wait comes near it)
+// also gives up when the device status word holds an error: once one CTA has
+// timed out, the CTAs still to come do not each spend a whole budget.
 struct WaitCtl {
     volatile int* abort_flag;   // shared memory
     uint64_t budget_ns;
     int* status;                // device status word of the library (global memory)
 };
 
+constexpr uint64_t kStatusPollNs = 1000000ull;   // 1 ms
+
 __device__ __forceinline__ bool wait_expired(const WaitCtl& w, uint64_t t0) {
     if (*w.abort_flag) return true;
-    if (global_timer_ns() - t0 > w.budget_ns) {
+    const uint64_t waited = global_timer_ns() - t0;
+    if (waited > w.budget_ns) {
         *w.abort_flag = 1;
         report_status(w.status, kStatusTimeout);
+        return true;
+    }
+    if (waited > kStatusPollNs && w.budget_ns > kStatusPollNs && *reinterpret_cast<volatile int*>(w.status) != 0) {
+        *w.abort_flag = 1;
         return true;
     }
     return false;
@@ -387,6 +397,15 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -400,6 +419,22 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
+}
+
+// 2^x for a pair, for results that are rounded to e4m3 next (3 mantissa bits): the same
+// range split as exp2_poly3 with a degree-2 minimax polynomial from
+// video_dit_full_b200/fit_exp2_poly.py --degree 2 (max relative error 1.73e-3, a
+// thirty-sixth of e4m3's half step), in packed pair arithmetic.  Clamped at -125 as above.
+__device__ __forceinline__ float2 exp2_poly2_x2(float2 x) {
+    x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+    const float2 magic = make_float2(12582912.f, 12582912.f);
+    const float2 j = fadd2(x, magic);                       // n in the low mantissa bits
+    const float2 f = fsub2(x, fsub2(j, magic));             // exact: x - n
+    float2 p = ffma2(make_float2(0.2384272813796997f, 0.2384272813796997f), f,
+                     make_float2(0.7034459114074707f, 0.7034459114074707f));
+    p = ffma2(p, f, make_float2(1.0004431009292603f, 1.0004431009292603f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
 }
 
 // Two floats -> packed bf16x2, round to nearest even; `lo` lands in the low half.
