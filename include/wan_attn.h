@@ -160,11 +160,12 @@ WAN_ATTN_API int wan_attn_cross_bwd(const void* q, const void* k, const void* v,
  *     at least wan_attn_fwd_block_sparse_workspace_size bytes: the per-CTA
  *     lists of attended key blocks (int32 [B, H, ceil(Sq/256), ceil(Skv/64)])
  *     and their lengths, built on the device by this call.
- * Work: a CTA covers 256 queries (4 query blocks) and runs its 128-row MMAs
- * over the union of the key blocks its 4 query blocks attend, two blocks per
- * step; the softmax masks each row to its own blocks.  With an all-ones mask
- * the result equals wan_attn_fwd bit for bit.  Other conventions as
- * wan_attn_fwd.
+ * Work: a CTA covers 256 queries (4 query blocks, two 128-row Q tiles) and
+ * streams the union of the key blocks its 4 query blocks attend, two blocks
+ * per step; each Q tile's MMAs cover only the blocks its own 2 query blocks
+ * attend (a 64-key half at a time), and the softmax masks each row to its own
+ * blocks.  With an all-ones mask the result equals wan_attn_fwd bit for bit.
+ * Other conventions as wan_attn_fwd.
  */
 WAN_ATTN_API size_t wan_attn_fwd_block_sparse_workspace_size(int B, int Sq, int Skv, int H, int D);
 WAN_ATTN_API int wan_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,

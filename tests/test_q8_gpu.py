@@ -87,6 +87,31 @@ def test_q8_720p_sampled_rows():
     check(x, rows=synth.sample_rows(w.S, 256))
 
 
+def test_q8_increasing_scores_rescale_every_block():
+    # s_ij = j / 20: each row's max rises by ~4.6 (log2 units) per 64-key block, so the running
+    # max moves at every block, the last (short) one included, and O is rescaled after every P V:
+    # the rescale's wait for the previous product runs on every step, through S(j + 1)'s barrier
+    # and, at the last block, the one-time barrier.  Against the recipe's simulation: P of the
+    # last block is quantised against the same max (up to an exact power of two) and earlier
+    # blocks weigh <= 2^-4.6 each, so the two agree far inside the recipe's own error.
+    B, S, H, D = 1, 1500, 1, 128
+    u = np.ones(D) / np.sqrt(D) * 4.0
+    q = np.broadcast_to(u, (B, S, H, D))
+    ramp = (np.arange(S) / 20.0)[None, :, None, None]
+    k = ramp * np.broadcast_to(u, (B, S, H, D)) * np.sqrt(D) / 16.0
+    v = np.random.default_rng(6).standard_normal((B, S, H, D))
+    x = {n: synth.f64_to_bf16_bits(a) for n, a in (("q", q), ("k", k), ("v", v))}
+    o, lse, _ = run_q8(x)
+    sim_o, sim_lse = quant8.attn_fwd_q8_sim(x["q"], x["k"], x["v"])
+    got = bf16_to_f64(o)
+    assert np.all(np.isfinite(got))
+    _, rel = errors(got, sim_o)
+    lse_err = float(np.abs(lse.cpu().numpy().astype(np.float64) - sim_lse).max())
+    print(f"q8 ramp: O rel-frob vs recipe {rel:.3e}, LSE {lse_err:.3e}")
+    assert rel <= 1e-2, rel
+    assert lse_err <= 3e-3, lse_err                # polynomial exponentials: ln(1 + 1.73e-3)
+
+
 def test_q8_uniform_scores_give_mean_of_dequantised_v():
     B, S, H = 1, 700, 2
     x = inputs_for(B, S, H, seed=9)

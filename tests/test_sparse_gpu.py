@@ -92,3 +92,23 @@ def test_720p_at_one_eighth_density_sampled_rows():
     nb = bs.blocks(w.S)
     mask = synth.block_mask(w.B, w.H, nb, nb, 0.125, seed=0)
     check(x, mask, rows=synth.sample_rows(w.S, 256))
+
+
+def test_tiles_that_need_one_half_or_start_late():
+    # Each CTA's tiles (query blocks 0-1 and 2-3 of its four) get their own MMAs:
+    # head 0: tile 0 attends even key blocks, tile 1 odd ones, so every step's two blocks split
+    #         between the tiles and each tile runs one 64-key half of it;
+    # head 1: tile 1 attends key blocks 0-2 only, tile 0 blocks 12.. only, the short last one
+    #         included, so tile 0 has no product for its first step and later steps start it.
+    B, H, S = 1, 2, 1500
+    x = inputs_for_cross(B, S, S, H, seed=12)
+    nb = bs.blocks(S)
+    mask = np.zeros((B, H, nb, nb), dtype=np.uint8)
+    for qb in range(nb):
+        tile = (qb % 4) // 2
+        mask[0, 0, qb, tile::2] = 1
+        if tile == 0:
+            mask[0, 1, qb, 12:] = 1
+        else:
+            mask[0, 1, qb, :3] = 1
+    check(x, mask)

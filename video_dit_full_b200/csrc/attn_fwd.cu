@@ -56,6 +56,10 @@ constexpr int SMEM_USED = OFF_ABORT + 8;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;   // slack for 1024-byte alignment of the tiles
 constexpr int NTHREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;            // S0 S1 O0 O1, 128 columns each
+// Sparse list entries: the key block in the low bits, and whether Q tile 0 / 1 of the CTA (its
+// query blocks 0-1 / 2-3) attends it in bits 28 / 29.
+constexpr int KB_BITS = (1 << 28) - 1;
+constexpr int NEED_SHIFT = 28;
 constexpr float RESCALE_THRESHOLD = 8.0f;      // log2 units: keep a stale max while p <= 2^8
 
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem, uint32_t idesc) {
@@ -68,14 +72,15 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint3
     }
 }
 
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc,
-                                         bool accumulate) {
-    // A = P (128 x 128 bf16 in TMEM, 2 per column), B = V stored [key][d] (MN-major):
-    // 16 keys per step = 2048 bytes; the two 64-wide halves of d are 16 KB apart (LBO).
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk) {
+// O += P V over the 16-key steps [kk0, kk1) of the tile (0-4: the first 64 keys, 4-8: the
+// second).  A = P (128 x 128 bf16 in TMEM, 2 per column), B = V stored [key][d] (MN-major):
+// 16 keys per step = 2048 bytes; the two 64-wide halves of d are 16 KB apart (LBO).  The first
+// MMA accumulates onto O only if `accumulate`.
+__device__ __forceinline__ void issue_pv_keys(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc,
+                                              bool accumulate, int kk0, int kk1) {
+    for (int kk = kk0; kk < kk1; ++kk) {
         mma_f16_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(v_smem + kk * 2048, HALF_BYTES, 1024), idesc,
-                   (accumulate || kk > 0) ? 1u : 0u);
+                   (accumulate || kk > kk0) ? 1u : 0u);
     }
 }
 
@@ -156,7 +161,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if constexpr (SPARSE) {
                     // two 64-key blocks into rows 0-63 and 64-127 of both 64-wide halves of d (a missing
                     // second block repeats the first; the softmax masks it)
-                    const int ka = kv_list[2 * j] * 64, kb = kv_list[min(2 * j + 1, kv_count - 1)] * 64;
+                    const int ka = (kv_list[2 * j] & KB_BITS) * 64;
+                    const int kb = (kv_list[min(2 * j + 1, kv_count - 1)] & KB_BITS) * 64;
                     for (int e = 0; e < 2; ++e) {
                         const uint32_t dst = sK + s * TILE_BYTES + e * HALF_BYTES;
                         tma_load_4d_hint(dst, &tmk, bar(K_FULL + s), 64 * e, h, ka, b, keep);
@@ -171,7 +177,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar(V_FULL + s), TILE_BYTES);
                 if constexpr (SPARSE) {
-                    const int ka = kv_list[2 * j] * 64, kb = kv_list[min(2 * j + 1, kv_count - 1)] * 64;
+                    const int ka = (kv_list[2 * j] & KB_BITS) * 64;
+                    const int kb = (kv_list[min(2 * j + 1, kv_count - 1)] & KB_BITS) * 64;
                     for (int e = 0; e < 2; ++e) {
                         const uint32_t dst = sV + s * TILE_BYTES + e * HALF_BYTES;
                         tma_load_4d_hint(dst, &tmv, bar(V_FULL + s), 64 * e, h, ka, b, keep);
@@ -196,14 +203,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         // ------------------------------ MMA issuer --------------------------------
         if (lane == 0) {
             const uint32_t idesc_qk = make_idesc(1, 1, 1, 0, 0, BM, BN);
+            const uint32_t idesc_qk64 = make_idesc(1, 1, 1, 0, 0, BM, BN / 2);
             const uint32_t idesc_pv = make_idesc(1, 1, 1, 0, 1, BM, HD);
+            // Which 64-key halves of step j tile t needs: bit 0 the first block, bit 1 the second.
+            // Dense: both.  Sparse: a half none of the tile's query blocks attends is neither
+            // computed (Q K^T of the other half alone, N = 64) nor multiplied into O; its S is
+            // never read, since every row of the tile has it masked.  The barriers still pass
+            // every step, so phases stay in step with the softmax.
+            auto need = [&](int j, int t) -> uint32_t {
+                if constexpr (!SPARSE) return 3u;
+                const uint32_t ea = static_cast<uint32_t>(kv_list[2 * j]);
+                const uint32_t eb = 2 * j + 1 < kv_count ? static_cast<uint32_t>(kv_list[2 * j + 1]) : 0u;
+                return ((ea >> (NEED_SHIFT + t)) & 1u) | (((eb >> (NEED_SHIFT + t)) & 1u) << 1);
+            };
+            auto qk = [&](int t, uint32_t k_stage, uint32_t nd) {
+                const uint32_t d = tmem + t * BN, qs = sQ + t * TILE_BYTES;
+                if (nd == 3u) issue_qk(d, qs, k_stage, idesc_qk);
+                else if (nd == 1u) issue_qk(d, qs, k_stage, idesc_qk64);
+                else if (nd == 2u) issue_qk(d + BN / 2, qs, k_stage + HALF_BYTES / 2, idesc_qk64);
+            };
+            bool o_init[2] = {false, false};               // has a P V product written O yet
+            auto pv = [&](int t, uint32_t v_stage, uint32_t nd) {
+                if (nd == 0u) return;
+                issue_pv_keys(tmem + 256 + t * HD, tmem + t * BN, v_stage, idesc_pv, o_init[t],
+                              nd & 1u ? 0 : 4, nd & 2u ? 8 : 4);
+                o_init[t] = true;
+            };
             bool ok = nkv > 0;                           // sparse: a CTA may attend no key block
             for (int t = 0; t < nq && ok; ++t) ok = wait_thread(bar(Q_FULL + t), 0, wc);
             if (ok) ok = wait_thread(bar(K_FULL + 0), 0, wc);
             if (ok) {
                 tc_fence_after();
                 for (int t = 0; t < nq; ++t) {
-                    issue_qk(tmem + t * BN, sQ + t * TILE_BYTES, sK, idesc_qk);
+                    qk(t, sK, need(0, t));
                     mma_commit(bar(S_FULL + t));
                 }
                 mma_commit(bar(K_EMPTY + 0));
@@ -216,7 +248,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     ok = wait_thread(bar(P_FULL + t), j & 1, wc);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(tmem + 256 + t * HD, tmem + t * BN, sV + s * TILE_BYTES, idesc_pv, j > 0);
+                    pv(t, sV + s * TILE_BYTES, need(j, t));
                     if (j + 1 == nkv) mma_commit(bar(O_FINAL + t));
                     if (j + 1 < nkv) {
                         if (t == 0) {
@@ -224,7 +256,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                             if (!ok) break;
                             tc_fence_after();
                         }
-                        issue_qk(tmem + t * BN, sQ + t * TILE_BYTES, sK + s1 * TILE_BYTES, idesc_qk);
+                        qk(t, sK + s1 * TILE_BYTES, need(j + 1, t));
                         mma_commit(bar(S_FULL + t));
                     }
                 }
@@ -263,7 +295,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 // the two key blocks of this step: each half keeps its keys if the row's query block
                 // attends the block (and the keys exist); a missing second block is masked.  A
                 // warp's 32 rows lie in one 64-row query block, so lim0 and lim1 are warp-uniform.
-                const int kba = kv_list[2 * j], kbb = (2 * j + 1 < kv_count) ? kv_list[2 * j + 1] : -1;
+                const int kba = kv_list[2 * j] & KB_BITS;
+                const int kbb = (2 * j + 1 < kv_count) ? (kv_list[2 * j + 1] & KB_BITS) : -1;
                 const int qb = min(row, p.S - 1) / 64;
                 const uint8_t* mrow = p.mask + ((static_cast<size_t>(b) * p.H + h) * p.nqb + qb) * p.nkb;
                 lim0 = mrow[kba] ? min(64, p.Skv - 64 * kba) : 0;
@@ -416,11 +449,13 @@ __global__ void __launch_bounds__(256) sparse_lists_kernel(const uint8_t* __rest
         int n = 0;
         for (int k0 = 0; k0 < nkb; k0 += 32) {
             const int kb = k0 + lane;
-            bool any = false;
+            int tiles = 0;                                // bit t: Q tile t (query blocks 2t, 2t+1)
             if (kb < nkb)
-                for (int r = 0; r < nrows; ++r) any |= m[static_cast<long long>(r) * nkb + kb] != 0;
+                for (int r = 0; r < nrows; ++r)
+                    if (m[static_cast<long long>(r) * nkb + kb] != 0) tiles |= 1 << (r >> 1);
+            const bool any = tiles != 0;
             const unsigned bal = __ballot_sync(0xffffffffu, any);
-            if (any) out[n + __popc(bal & ((1u << lane) - 1u))] = kb;
+            if (any) out[n + __popc(bal & ((1u << lane) - 1u))] = kb | (tiles << NEED_SHIFT);
             n += __popc(bal);
         }
         if (lane == 0) count[w] = n;
