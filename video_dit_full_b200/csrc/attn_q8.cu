@@ -354,23 +354,19 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             const int kx = min(sv_max_exp - static_cast<int>(__float_as_uint(sv_cur) >> 23), 64);
             const float inv = __uint_as_float(static_cast<uint32_t>(127 + kx) << 23) * (1.f / P_SCALE);
             const float2 c2 = make_float2(c, c);
-            const float2 magic2 = make_float2(12582912.f, 12582912.f);
             uint32_t pk[16];
             float sum = 0.f, mx = -INFINITY;
             // One pass over the row's 64 scores of this block: P8 and the row sum against the
-            // max m, and with `with_max` the block's max.  int32 -> float without the
-            // conversion unit: |S| <= 128*127*127 < 2^22, so the bit pattern of S + 0x4B400000
-            // is the float 1.5*2^23 + S, exactly and in S's order (the max is taken over those
-            // floats); then xm - 1.5*2^23 = S exactly and s - bias = S c - bias in one fused
-            // multiply-add per pair.
+            // max m, and with `with_max` the block's max.  The int32 S converts to fp32 exactly
+            // (|S| <= 128*127*127 < 2^24); s - bias = S c - bias is one fused multiply-add per pair.
             uint32_t sr[64];
-            float* xm = reinterpret_cast<float*>(sr);
+            float* xm = reinterpret_cast<float*>(sr);     // S as fp32, in place
             auto load = [&]() {
                 tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                 tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 64; ++e) sr[e] += 0x4B400000u;
+                for (int e = 0; e < 64; ++e) xm[e] = __int2float_rn(static_cast<int>(sr[e]));
                 if (valid < BN) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e)
@@ -386,8 +382,8 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 for (int w = 0; w < 16; ++w) {
                     if (with_max)
                         m4[w & 3] = fmax3(fmax3(m4[w & 3], xm[4 * w], xm[4 * w + 1]), xm[4 * w + 2], xm[4 * w + 3]);
-                    const float2 x01 = ffma2(fsub2(make_float2(xm[4 * w], xm[4 * w + 1]), magic2), c2, n2);
-                    const float2 x23 = ffma2(fsub2(make_float2(xm[4 * w + 2], xm[4 * w + 3]), magic2), c2, n2);
+                    const float2 x01 = ffma2(make_float2(xm[4 * w], xm[4 * w + 1]), c2, n2);
+                    const float2 x23 = ffma2(make_float2(xm[4 * w + 2], xm[4 * w + 3]), c2, n2);
                     float2 p01, p23;
                     if ((w & 7) < Q8_POLY_GROUPS) {
                         p01 = exp2_poly2_x2(x01);
@@ -400,7 +396,7 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                     pk[w] = pack_e4m3x2(p01.x, p01.y) | (pack_e4m3x2(p23.x, p23.y) << 16);
                 }
                 sum = (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
-                if (with_max) mx = (fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) - 12582912.f) * c;
+                if (with_max) mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * c;
             };
             // P is computed against the max in use while the block's max is found in the same
             // pass; a row whose max moves is redone against the new max (warp-wide, as TMEM loads
@@ -420,7 +416,7 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                     for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], xm[e + q], xm[e + 4 + q]);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], xm[60 + q]);
-                mx = (fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) - 12582912.f) * c;
+                mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * c;
             }
 #endif
             float alpha = 1.f;
