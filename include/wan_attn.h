@@ -286,7 +286,10 @@ WAN_ATTN_API size_t wan_attn_fwd_q8_workspace_size(int B, int S, int H, int D);
  *     the head's largest V block scale: each block's V scale rides in P;
  *   - every block's P8 V8 is summed by the tensor core's fp32 accumulator
  *     (fp32 accumulation across blocks); O = that sum * sV_max / 224 / l,
- *     with the row sum l taken over the unquantised exponentials.
+ *     with the row sum l taken over the unquantised exponentials;
+ *   - exp is evaluated in fp32, for 3 in 8 of the scores by a degree-2
+ *     polynomial with relative error <= 1.73e-3 (below e4m3's half step),
+ *     so the LSE carries up to ln(1 + 1.73e-3) beyond the score error.
  *   q, k, v : in,  bf16 [B, S, H, D]
  *   o       : out, bf16 [B, S, H, D]
  *   lse     : out, fp32 [B, H, S], natural log, of the dequantised scores
