@@ -34,7 +34,7 @@ METRIC = "attention TFLOP/s (4*B*H*S^2*D fwd)"
 # DRAM bytes (read + write) of one launch of the dominant kernel from an ncu
 # capture (profiles/), per workload; None where the kernel changed since.
 TRAFFIC = {"wan14b_720p": 3.337e9, "train_480p_fwd_bwd": 3.809e9, "q8_720p": 1.936e9, "fp8_qkv_720p": 5.028e9,
-           "sparse8_720p": 3.538e9}
+           "sparse8_720p": 3.429e9}
 
 
 def load_peaks():

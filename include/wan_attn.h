@@ -157,15 +157,13 @@ WAN_ATTN_API int wan_attn_cross_bwd(const void* q, const void* k, const void* v,
  *   o : out bf16 [B, Sq, H, D];  lse : out fp32 [B, H, Sq]
  *   A row whose query block attends no key block gets o = 0 and lse = -inf.
  *   workspace, workspace_bytes : caller-owned device memory, 256-byte aligned,
- *     at least wan_attn_fwd_block_sparse_workspace_size bytes: the per-CTA
- *     lists of attended key blocks (int32 [B, H, ceil(Sq/256), ceil(Skv/64)])
+ *     at least wan_attn_fwd_block_sparse_workspace_size bytes: the per-tile
+ *     lists of attended key blocks (int32 [B, H, ceil(Sq/128), ceil(Skv/64)])
  *     and their lengths, built on the device by this call.
- * Work: a CTA covers 256 queries (4 query blocks, two 128-row Q tiles) and
- * streams the union of the key blocks its 4 query blocks attend, two blocks
- * per step; each Q tile's MMAs cover only the blocks its own 2 query blocks
- * attend (a 64-key half at a time), and the softmax masks each row to its own
- * blocks.  With an all-ones mask the result equals wan_attn_fwd bit for bit.
- * Other conventions as wan_attn_fwd.
+ * Work: a CTA covers one 128-row Q tile (2 query blocks) and steps through
+ * the union of the key blocks its 2 query blocks attend, one 64-key block per
+ * step; each row keeps only its own query block's blocks.  Other conventions
+ * as wan_attn_fwd.
  */
 WAN_ATTN_API size_t wan_attn_fwd_block_sparse_workspace_size(int B, int Sq, int Skv, int H, int D);
 WAN_ATTN_API int wan_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,

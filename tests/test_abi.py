@@ -140,10 +140,10 @@ def test_sparse_fp8_cp_host_side_validation_without_gpu(built):
     INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 5
     P = [ctypes.c_void_p(0x100000 + i * 0x10000000) for i in range(8)]
     q, k, v, o, lse, mask, ws, z = P
-    # block-sparse: lists int32 [B, H, ceil(Sq/256), ceil(Skv/64)] + lengths, each 256-byte aligned
+    # block-sparse: lists int32 [B, H, ceil(Sq/128), ceil(Skv/64)] + lengths, each 256-byte aligned
     need = lib.wan_attn_fwd_block_sparse_workspace_size(1, 300, 700, 2, 128)
     a = lambda x: (x + 255) // 256 * 256
-    assert need == a(2 * 2 * 11 * 4) + a(2 * 2 * 4)
+    assert need == a(2 * 3 * 11 * 4) + a(2 * 3 * 4)
     assert lib.wan_attn_fwd_block_sparse_workspace_size(1, 300, 700, 2, 96) == 0
     args = [q, k, v, o, lse, mask, 1, 300, 700, 2, 128, ws, need, None]
     assert lib.wan_attn_fwd_block_sparse(*args[:5], None, *args[6:]) == INVALID          # no mask

@@ -1,7 +1,8 @@
 """Parity of the block-sparse forward (wan_attn_fwd_block_sparse, through the C ABI) with the oracle
 (oracle/block_sparse.py): the bf16 forward's bars (O max-abs 1e-2 and rel-Frobenius 5e-3, LSE
 1e-3) on the rows that attend something; rows that attend nothing must be exactly O = 0,
-LSE = -inf.  An all-ones mask must reproduce wan_attn_fwd bit for bit (same arithmetic)."""
+LSE = -inf.  An all-ones mask must agree with wan_attn_fwd to rounding (the two kernels take
+the keys in steps of 64 and 128, so their online softmax rescales at different points)."""
 import numpy as np
 import pytest
 
@@ -45,16 +46,20 @@ def check(x, mask, rows=None, heads=None):
         assert lse_err <= LSE_MAX_ABS, lse_err
 
 
-def test_all_ones_mask_is_the_dense_call_bit_for_bit():
-    import torch
+def test_all_ones_mask_matches_the_dense_call():
     import video_dit_full_b200 as wa
     x = inputs_for_cross(2, 1000, 1000, 3, seed=21)
     mask = np.ones((2, 3, bs.blocks(1000), bs.blocks(1000)), dtype=np.uint8)
+    check(x, mask)
     o, lse = run(x, mask)
     q, k, v = (to_device(x[n]) for n in "qkv")
     od, ld = wa.fwd(q, k, v)
     wa.check_status()
-    assert torch.equal(o, od) and torch.equal(lse, ld)
+    # each call is within the forward's bars of the exact result (bf16 output rounding, ~2.3e-3
+    # rel-Frobenius apiece), so the two are within the sum of those bars of each other
+    max_abs, rel = errors(bf16_to_f64(o), bf16_to_f64(od))
+    assert rel <= 2 * O_REL_FROB and max_abs <= 2 * O_MAX_ABS, (rel, max_abs)
+    assert float((lse - ld).abs().max()) <= 2 * LSE_MAX_ABS
 
 
 @pytest.mark.parametrize("Sq,Skv,keep", [(1000, 1000, 0.5), (1000, 1000, 0.125), (300, 777, 0.25),

@@ -221,12 +221,12 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     return launch_fwd(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
 }
 
-// Block-sparse forward: per CTA (2 Q tiles = 4 query blocks of 64) the list of attended key
-// blocks, int32 [B, H, nctas, nkb], then the lists' lengths [B, H, nctas].
+// Block-sparse forward: per 128-row Q tile (2 query blocks of 64) the list of attended key
+// blocks, int32 [B, H, ntiles, nkb], then the lists' lengths [B, H, ntiles].
 size_t sparse_ws_size(int B, int Sq, int Skv, int H, int D) {
     if (check_shape(B, Sq, H, D) != WAN_ATTN_OK || check_shape(B, Skv, H, D) != WAN_ATTN_OK) return 0;
-    const size_t nctas = (size_t(Sq) + 255) / 256, nkb = (size_t(Skv) + 63) / 64;
-    return align256(size_t(B) * H * nctas * nkb * 4) + align256(size_t(B) * H * nctas * 4);
+    const size_t ntiles = (size_t(Sq) + 127) / 128, nkb = (size_t(Skv) + 63) / 64;
+    return align256(size_t(B) * H * ntiles * nkb * 4) + align256(size_t(B) * H * ntiles * 4);
 }
 
 int fwd_block_sparse_impl(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* mask,
@@ -241,7 +241,7 @@ int fwd_block_sparse_impl(const void* q, const void* k, const void* v, void* o, 
     const size_t need = sparse_ws_size(B, Sq, Skv, H, D);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return WAN_ATTN_ERR_WORKSPACE;
-    const int nqb = (Sq + 63) / 64, nkb = (Skv + 63) / 64, nctas = (Sq + 255) / 256;
+    const int nqb = (Sq + 63) / 64, nkb = (Skv + 63) / 64, ntiles = (Sq + 127) / 128;
     const size_t nq = size_t(B) * Sq * H * D, nkv = size_t(B) * Skv * H * D;
     const Range ins[] = {range_of(q, nq * 2), range_of(k, nkv * 2), range_of(v, nkv * 2),
                          range_of(mask, size_t(B) * H * nqb * nkb)};
@@ -266,16 +266,16 @@ int fwd_block_sparse_impl(const void* q, const void* k, const void* v, void* o, 
     p.mask = mask;
     p.kv_list = static_cast<const int*>(workspace);
     p.kv_count = reinterpret_cast<const int*>(static_cast<char*>(workspace) +
-                                              align256(size_t(B) * H * nctas * nkb * 4));
+                                              align256(size_t(B) * H * ntiles * nkb * 4));
     p.nqb = nqb;
     p.nkb = nkb;
-    p.nctas = nctas;
+    p.nctas = ntiles;
     p.scale_log2 = static_cast<float>((1.0 / std::sqrt(double(D))) * 1.4426950408889634);
     p.wait_budget_ns = wait_budget_ns();
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
-    return launch_fwd_block_sparse(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
-                                                                                       : WAN_ATTN_ERR_CUDA;
+    return launch_fwd_block_sparse_tiles(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                             : WAN_ATTN_ERR_CUDA;
 }
 
 // Backward workspace: fp32 dQ accumulator [B, Sq, H, D], fp32 D_i [B, H, Sq] and, for the

@@ -14,9 +14,10 @@ struct FwdParams {
     float* lse;                 // fp32 [B, H, S], natural log
     int B, S, H;                // S = query tokens
     int Skv;                    // key / value tokens (= S for self-attention)
-    // block-sparse forward only: 64 x 64 block mask uint8 [B, H, nqb, nkb], and per CTA (2 Q
-    // tiles = 4 query blocks) the ascending list of key blocks any of them attends
-    // (kv_list [B, H, nctas, nkb] int32) with its length (kv_count [B, H, nctas])
+    // block-sparse forward only: 64 x 64 block mask uint8 [B, H, nqb, nkb], and per 128-row Q
+    // tile (2 query blocks) the ascending list of key blocks either attends
+    // (kv_list [B, H, nctas, nkb] int32, nctas = the number of Q tiles) with its length
+    // (kv_count [B, H, nctas])
     const uint8_t* mask;
     const int* kv_list;
     const int* kv_count;
@@ -78,10 +79,11 @@ int configure_smem(const void* kernel, int bytes);
 
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                cudaStream_t stream);
-// Block-sparse forward: tk64 / tv64 are K / V maps with 64-token boxes.  Builds the key-block
-// lists in p.kv_list / p.kv_count (device workspace), then runs the sparse kernel.
-int launch_fwd_block_sparse(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64,
-                            const FwdParams& p, cudaStream_t stream);
+// Block-sparse forward, one CTA per 128-row Q tile (p.nctas = the number of Q tiles); tk64 / tv64
+// are K / V maps with 64-token boxes.  Builds each tile's key-block list in p.kv_list /
+// p.kv_count (device workspace), then runs the sparse kernel.
+int launch_fwd_block_sparse_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64,
+                                  const FwdParams& p, cudaStream_t stream);
 
 // Chooses p.nsplit (1 unless allow_split and the key tiles alone fill too few waves of the
 // GPU), then launches the backward's kernels.  tdk / tdv (fp32 accumulators, as tdq) are only
