@@ -62,8 +62,11 @@ def test_all_ones_mask_matches_the_dense_call():
     assert float((lse - ld).abs().max()) <= 2 * LSE_MAX_ABS
 
 
+# (1, 1), (129, 64): one key block, a single step; (200, 100): two steps, the next-to-last
+# product's barrier at step 0; (300, 130): three steps, the last one short
 @pytest.mark.parametrize("Sq,Skv,keep", [(1000, 1000, 0.5), (1000, 1000, 0.125), (300, 777, 0.25),
-                                         (4100, 4100, 0.125), (65, 64, 1.0)])
+                                         (4100, 4100, 0.125), (65, 64, 1.0), (1, 1, 1.0), (129, 64, 1.0),
+                                         (200, 100, 1.0), (300, 130, 1.0)])
 def test_random_masks(Sq, Skv, keep):
     B, H = 1, 2
     x = inputs_for_cross(B, Sq, Skv, H, seed=Sq + Skv)
