@@ -354,71 +354,30 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             const int kx = min(sv_max_exp - static_cast<int>(__float_as_uint(sv_cur) >> 23), 64);
             const float inv = __uint_as_float(static_cast<uint32_t>(127 + kx) << 23) * (1.f / P_SCALE);
             const float2 c2 = make_float2(c, c);
-            uint32_t pk[16];
-            float sum = 0.f, mx = -INFINITY;
-            // One pass over the row's 64 scores of this block: P8 and the row sum against the
-            // max m, and with `with_max` the block's max.  The int32 S converts to fp32 exactly
-            // (|S| <= 128*127*127 < 2^24); s - bias = S c - bias is one fused multiply-add per pair.
+            // S: the int32 sums convert to fp32 exactly (|S| <= 128*127*127 < 2^24), keys past S
+            // masked; the block's max
             uint32_t sr[64];
             float* xm = reinterpret_cast<float*>(sr);     // S as fp32, in place
-            auto load = [&]() {
-                tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_wait_ld();
+            tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 64; ++e) xm[e] = __int2float_rn(static_cast<int>(sr[e]));
-                if (valid < BN) {
+            for (int e = 0; e < 64; ++e) xm[e] = __int2float_rn(static_cast<int>(sr[e]));
+            if (valid < BN) {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e)
-                        if (e >= valid) xm[e] = -INFINITY;
-                }
-            };
-            auto pass = [&](float m, bool with_max) {
-                const float nb = -(m - (LOG2_P_SCALE - static_cast<float>(kx)));
-                const float2 n2 = make_float2(nb, nb);
-                float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int w = 0; w < 16; ++w) {
-                    if (with_max)
-                        m4[w & 3] = fmax3(fmax3(m4[w & 3], xm[4 * w], xm[4 * w + 1]), xm[4 * w + 2], xm[4 * w + 3]);
-                    const float2 x01 = ffma2(make_float2(xm[4 * w], xm[4 * w + 1]), c2, n2);
-                    const float2 x23 = ffma2(make_float2(xm[4 * w + 2], xm[4 * w + 3]), c2, n2);
-                    float2 p01, p23;
-                    if ((w & 7) < Q8_POLY_GROUPS) {
-                        p01 = exp2_poly2_x2(x01);
-                        p23 = exp2_poly2_x2(x23);
-                    } else {
-                        p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
-                        p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-                    }
-                    sum2[w & 1] = fadd2(sum2[w & 1], fadd2(p01, p23));
-                    pk[w] = pack_e4m3x2(p01.x, p01.y) | (pack_e4m3x2(p23.x, p23.y) << 16);
-                }
-                sum = (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
-                if (with_max) mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * c;
-            };
-            // P is computed against the max in use while the block's max is found in the same
-            // pass; a row whose max moves is redone against the new max (warp-wide, as TMEM loads
-            // are; after the first few blocks this is rare, and the first block always is).
-#if WAN_Q8_SPECULATE
-            load();
-            pass(m_ref, true);
-#else
-            load();
-            {
-                float m4[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) m4[q] = fmax3(xm[q], xm[q + 4], xm[q + 8]);
-#pragma unroll
-                for (int e = 12; e + 8 <= 64; e += 8)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], xm[e + q], xm[e + 4 + q]);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], xm[60 + q]);
-                mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * c;
+                for (int e = 0; e < 64; ++e)
+                    if (e >= valid) xm[e] = -INFINITY;
             }
-#endif
+            float m4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) m4[q] = fmax3(xm[q], xm[q + 4], xm[q + 8]);
+#pragma unroll
+            for (int e = 12; e + 8 <= 64; e += 8)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) m4[q] = fmax3(m4[q], xm[e + q], xm[e + 4 + q]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], xm[60 + q]);
+            const float mx = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * c;
             float alpha = 1.f;
             bool moved = false;
             if (mx > m_ref + RESCALE_THRESHOLD) {
@@ -427,14 +386,27 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 moved = true;
             }
             const bool any_moved = __any_sync(0xffffffffu, moved);
-#if WAN_Q8_SPECULATE
-            if (any_moved) {
-                load();
-                pass(m_ref, false);
+            // P8 and the row sum: s - bias = S c - bias in one fused multiply-add per pair
+            const float nb = -(m_ref - (LOG2_P_SCALE - static_cast<float>(kx)));
+            const float2 n2 = make_float2(nb, nb);
+            float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            uint32_t pk[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                const float2 x01 = ffma2(make_float2(xm[4 * w], xm[4 * w + 1]), c2, n2);
+                const float2 x23 = ffma2(make_float2(xm[4 * w + 2], xm[4 * w + 3]), c2, n2);
+                float2 p01, p23;
+                if ((w & 7) < Q8_POLY_GROUPS) {
+                    p01 = exp2_poly2_x2(x01);
+                    p23 = exp2_poly2_x2(x23);
+                } else {
+                    p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+                    p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+                }
+                sum2[w & 1] = fadd2(sum2[w & 1], fadd2(p01, p23));
+                pk[w] = pack_e4m3x2(p01.x, p01.y) | (pack_e4m3x2(p23.x, p23.y) << 16);
             }
-#else
-            pass(m_ref, false);
-#endif
+            const float sum = (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
             tmem_st16(tS, pk);                                   // P8 over S's first 16 columns
             // the row sum counts p itself: scale by 1 / (P_SCALE * r_blk) = 2^k / P_SCALE
             l = l * alpha + sum * inv;
