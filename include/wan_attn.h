@@ -112,7 +112,9 @@ WAN_ATTN_API int wan_attn_bwd(const void* q, const void* k, const void* v, const
  * No mask: the Skv keys are all attended to (a caller whose text is padded
  * passes the padded embedding, as the 512-token condition is).  Other
  * conventions, precision and errors as wan_attn_fwd; wan_attn_cross_fwd with
- * Skv = Sq and the same pointers computes what wan_attn_fwd does.
+ * Skv = Sq and the same pointers computes what wan_attn_fwd does, bit for bit.
+ * With Sq != Skv <= 1024 the call takes 64 keys per step (one CTA per
+ * 128-query tile, two per SM), so its rounding differs from a 128-key step's.
  */
 WAN_ATTN_API int wan_attn_cross_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                                     int Sq, int Skv, int H, int D, void* stream);

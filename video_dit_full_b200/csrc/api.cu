@@ -187,9 +187,12 @@ using namespace wan;
 
 namespace {
 
-// Forward of Sq queries against Skv keys (self-attention: Skv = Sq).
+// Forward of Sq queries against Skv keys (self-attention: Skv = Sq).  The cross-attention call
+// with a short key sequence (Skv <= 1024, Sq != Skv: the text embedding) runs the per-tile
+// kernel: with a few key blocks per tile, a CTA's prologue and epilogue are much of its time,
+// and two CTAs per SM hide each other's.
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq, int Skv, int H,
-             int D, void* stream) {
+             int D, void* stream, bool cross) {
     if (!q || !k || !v || !o || !lse) return WAN_ATTN_ERR_INVALID_ARG;
     int st = check_shape(B, Sq, H, D);
     if (st == WAN_ATTN_OK) st = check_shape(B, Skv, H, D);
@@ -203,9 +206,11 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
         if (overlaps(ro, in) || overlaps(rl, in)) return WAN_ATTN_ERR_INVALID_ARG;
     if (overlaps(ro, rl)) return WAN_ATTN_ERR_INVALID_ARG;
 
+    const bool per_tile = cross && Sq != Skv && Skv <= 1024;
+    const int kv_box = per_tile ? 64 : 128;
     CUtensorMap tq, tk, tv;
-    if (!make_bshd_map(&tq, q, B, Sq, H, D, 128) || !make_bshd_map(&tk, k, B, Skv, H, D, 128) ||
-        !make_bshd_map(&tv, v, B, Skv, H, D, 128))
+    if (!make_bshd_map(&tq, q, B, Sq, H, D, 128) || !make_bshd_map(&tk, k, B, Skv, H, D, kv_box) ||
+        !make_bshd_map(&tv, v, B, Skv, H, D, kv_box))
         return WAN_ATTN_ERR_CUDA;
     FwdParams p{};
     p.o = o;
@@ -218,6 +223,13 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.wait_budget_ns = wait_budget_ns();
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
+    if (per_tile) {
+        p.nqb = (Sq + 63) / 64;
+        p.nkb = (Skv + 63) / 64;
+        p.nctas = (Sq + 127) / 128;
+        return launch_fwd_tiles(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                       : WAN_ATTN_ERR_CUDA;
+    }
     return launch_fwd(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
 }
 
@@ -274,8 +286,8 @@ int fwd_block_sparse_impl(const void* q, const void* k, const void* v, void* o, 
     p.wait_budget_ns = wait_budget_ns();
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
-    return launch_fwd_block_sparse_tiles(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
-                                                                                             : WAN_ATTN_ERR_CUDA;
+    return launch_fwd_tiles(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                   : WAN_ATTN_ERR_CUDA;
 }
 
 // Backward workspace: fp32 dQ accumulator [B, Sq, H, D], fp32 D_i [B, H, Sq] and, for the
@@ -358,12 +370,12 @@ extern "C" {
 
 int wan_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S, int H, int D,
                  void* stream) {
-    return fwd_impl(q, k, v, o, lse, B, S, S, H, D, stream);
+    return fwd_impl(q, k, v, o, lse, B, S, S, H, D, stream, false);
 }
 
 int wan_attn_cross_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq, int Skv,
                        int H, int D, void* stream) {
-    return fwd_impl(q, k, v, o, lse, B, Sq, Skv, H, D, stream);
+    return fwd_impl(q, k, v, o, lse, B, Sq, Skv, H, D, stream, true);
 }
 
 size_t wan_attn_bwd_workspace_size(int B, int S, int H, int D) { return bwd_ws_size(B, S, S, H, D, false); }

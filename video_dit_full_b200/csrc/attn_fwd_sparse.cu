@@ -6,6 +6,11 @@
 // scaling runs) and compares against FlexAttention on the same 64 x 64 block-sparse mask.
 // The mask is an input here; the learned coarse stage that picks the blocks is not built.
 //
+// Without a list (p.kv_list null) the same kernel steps through every key block: the
+// cross-attention to the short text embedding ("Wan 2.1 ... paper-podcast summary", section
+// "干预与形式化": cross-attention from the video tokens to the umT5 text tokens) takes it, since
+// at a few key blocks per tile two CTAs per SM hide each other's prologue and epilogue.
+//
 // How (one CTA = one 128-row Q tile = 2 query blocks of one (b, h); two CTAs per SM, each
 // with half of the tensor memory):
 //   sparse_tile_lists  one warp per (b, h, Q tile): the ascending union of the key blocks
@@ -87,8 +92,10 @@ attn_fwd_sparse_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_con
     const int h = blockIdx.y, b = blockIdx.z;
     const int q0 = blockIdx.x * BM;
     const size_t li = (static_cast<size_t>(b) * p.H + h) * p.nctas + blockIdx.x;
-    const int* list = p.kv_list + li * p.nkb;
-    const int n = p.kv_count[li];                    // key blocks this tile attends
+    const bool dense = p.kv_list == nullptr;         // every key block, no mask
+    const int* list = dense ? nullptr : p.kv_list + li * p.nkb;
+    const int n = dense ? p.nkb : p.kv_count[li];    // key blocks this tile attends
+    auto block_of = [&](int k) { return dense ? k : list[k]; };
 
     const uint32_t sQ = base + OFF_Q, sK = base + OFF_K, sV = base + OFF_V;
     const uint32_t bar0 = base + OFF_BAR;
@@ -135,7 +142,7 @@ attn_fwd_sparse_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_con
             bool ok = true;
             for (int k = 0; k < n && ok; ++k) {
                 const int s = k & 1, use = (k >> 1) & 1;
-                const int key0 = list[k] * BK;
+                const int key0 = block_of(k) * BK;
                 ok = wait_thread(bar(K_EMPTY + s), use ^ 1, wc);
                 if (!ok) break;
                 mbar_arrive_expect_tx(bar(K_FULL + s), KV_BYTES);
@@ -203,14 +210,15 @@ attn_fwd_sparse_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_con
         const int row = q0 + r;
         const float c = p.scale_log2;
         // the row's query block (the same for the warp's 32 rows; rows past S use the last one)
-        const uint8_t* mrow = p.mask + ((static_cast<size_t>(b) * p.H + h) * p.nqb + min(row, p.S - 1) / 64) * p.nkb;
+        const uint8_t* mrow =
+            dense ? nullptr : p.mask + ((static_cast<size_t>(b) * p.H + h) * p.nqb + min(row, p.S - 1) / 64) * p.nkb;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         // keys of step k this row keeps (0: its query block does not attend the step's key block;
         // short for the last key block); read one step ahead
         auto keep_of = [&](int k) {
-            const int kb = list[k];
-            return mrow[kb] ? min(BK, p.Skv - BK * kb) : 0;
+            const int kb = block_of(k);
+            return (dense || mrow[kb]) ? min(BK, p.Skv - BK * kb) : 0;
         };
         int lim_next = n > 0 ? keep_of(0) : 0;
         for (int k = 0; k < n && ok; ++k) {
@@ -358,15 +366,17 @@ __global__ void __launch_bounds__(256) sparse_tile_lists_kernel(const uint8_t* _
 
 }  // namespace sparse
 
-int launch_fwd_block_sparse_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64,
-                                  const FwdParams& p, cudaStream_t stream) {
-    int sms = 148, dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long long nlists = static_cast<long long>(p.B) * p.H * p.nctas;
-    sparse::sparse_tile_lists_kernel<<<sms * 8, 256, 0, stream>>>(p.mask, const_cast<int*>(p.kv_list),
-                                                                  const_cast<int*>(p.kv_count), nlists, p.nctas,
-                                                                  p.nqb, p.nkb);
-    if (cudaGetLastError() != cudaSuccess) return -1;
+int launch_fwd_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64, const FwdParams& p,
+                     cudaStream_t stream) {
+    if (p.kv_list) {
+        int sms = 148, dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const long long nlists = static_cast<long long>(p.B) * p.H * p.nctas;
+        sparse::sparse_tile_lists_kernel<<<sms * 8, 256, 0, stream>>>(p.mask, const_cast<int*>(p.kv_list),
+                                                                      const_cast<int*>(p.kv_count), nlists, p.nctas,
+                                                                      p.nqb, p.nkb);
+        if (cudaGetLastError() != cudaSuccess) return -1;
+    }
     if (configure_smem(reinterpret_cast<const void*>(sparse::attn_fwd_sparse_kernel), sparse::SMEM_BYTES) != 0)
         return -1;
     const dim3 grid(p.nctas, p.H, p.B);

@@ -79,11 +79,12 @@ int configure_smem(const void* kernel, int bytes);
 
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                cudaStream_t stream);
-// Block-sparse forward, one CTA per 128-row Q tile (p.nctas = the number of Q tiles); tk64 / tv64
-// are K / V maps with 64-token boxes.  Builds each tile's key-block list in p.kv_list /
-// p.kv_count (device workspace), then runs the sparse kernel.
-int launch_fwd_block_sparse_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64,
-                                  const FwdParams& p, cudaStream_t stream);
+// Forward with one CTA per 128-row Q tile (p.nctas = the number of Q tiles), 64-key steps; tk64 /
+// tv64 are K / V maps with 64-token boxes.  Block-sparse (p.kv_list set): builds each tile's
+// key-block list in p.kv_list / p.kv_count (device workspace) from p.mask, then runs the kernel
+// over the lists.  p.kv_list null: every key block, no mask.
+int launch_fwd_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64, const FwdParams& p,
+                     cudaStream_t stream);
 
 // Chooses p.nsplit (1 unless allow_split and the key tiles alone fill too few waves of the
 // GPU), then launches the backward's kernels.  tdk / tdv (fp32 accumulators, as tdq) are only
