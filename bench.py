@@ -281,7 +281,10 @@ class Path:
         else:
             self.flop = w.fwd_flop
             self.dominant_flop = w.fwd_flop
-            self.kernel = "wan::fwd::attn_fwd_kernel" + (" (wan_attn_cross_fwd)" if w.cross else "")
+            if w.cross and w.kv_len != w.S and w.kv_len <= 1024:   # the short-key cross forward's kernel
+                self.kernel = "wan::sparse::attn_fwd_sparse_kernel, every key block (wan_attn_cross_fwd)"
+            else:
+                self.kernel = "wan::fwd::attn_fwd_kernel" + (" (wan_attn_cross_fwd)" if w.cross else "")
             self.launches_per_step = 1
             self.peak_key, self.dtype = "bf16", "bf16"
         self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
@@ -495,7 +498,8 @@ class SparsePath:
                               device=dev)
         self.outs = [self.o, self.lse]
         self.dominant_flop = self.flop
-        self.kernel = "wan::fwd::attn_fwd_kernel<true> (with its key-block list kernel: one wan_attn_fwd_block_sparse)"
+        self.kernel = ("wan::sparse::attn_fwd_sparse_kernel (with its per-tile key-block list kernel: one "
+                       "wan_attn_fwd_block_sparse)")
         self.launches_per_step = 2
         self.peak_key, self.dtype = "bf16", "bf16"
         self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
