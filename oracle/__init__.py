@@ -6,11 +6,15 @@ CPU-baseline leg of ``bench.py`` are its only users.  The product path
 nothing here imports the product path; the two share only the seeded input
 generator in ``synth``.
 
-Parity pins: every function here is checked in ``tests/test_oracle.py``
+Parity pins: every function here is checked in ``tests/test_oracle*.py``
 against brute force, closed forms, invariants and finite differences (see
-that file).  ``quant8.attn_fwd_q8_sim`` is a diagnostic whose assembly is
-"parity unpinned" (its quantisers are pinned; the 8-bit path's gate is the
-unquantised ``attention.attn_fwd``).
+those files).  The 8-bit recipe is simulated in two independent forms:
+``quant8.attn_fwd_q8_sim`` (each block's V scale folded into P, one
+accumulation) and ``quant8.attn_fwd_q8_blockwise`` (each block's 8-bit product
+dequantised on its own and accumulated across blocks).  They are pinned to each
+other (equal wherever no P code is subnormal), to the uniform-score closed form
+and to the exact oracle's error budget; the 8-bit path's parity gate is the
+unquantised ``attention.attn_fwd``.
 """
 from .attention import attn_bwd, attn_fwd, softmax_matrix, widen  # noqa: F401
 from . import quant8  # noqa: F401

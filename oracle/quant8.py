@@ -118,15 +118,26 @@ def quant_e4m3(x, block: int = BLOCK):
     return e4m3_bits(quot), e4m3_round(quot), scale
 
 
+def _fold_factor(sv_bh: np.ndarray, S: int, block: int) -> np.ndarray:
+    """Per key j of one (b, h): sV(t(j)) / sV_max, the power-of-two factor that carries the
+    key's 64-token block scale into P in the folded form of the recipe."""
+    sv_key = np.repeat(sv_bh, block)[:S].astype(np.float64)
+    return sv_key / float(sv_bh.max())
+
+
 def attn_fwd_q8_sim(q, k, v, rows=None, heads=None, block: int = BLOCK):
-    """Diagnostic fp64 simulation of the 8-bit recipe (not a parity gate).
+    """Diagnostic fp64 simulation of the 8-bit recipe in its folded form.
 
     Scores from the int8 codes, s_ij = (q8_i . k8_j) sQ(i) sK(j) / sqrt(D);
     p_ij = exp(s_ij - max_j s_ij) in [0, 1]; l_i = sum_j p_ij (unquantised).
     Each 64-key block t's V scale is folded into P before P is quantised,
     P8_ij = e4m3(448 p_ij sV(t) / sV_max) with sV_max the largest block scale
     of the (b, h), so one fp32 accumulation carries every block:
-    o_i = (sum_j P8_ij v8_j) * sV_max / 448 / l_i."""
+    o_i = (sum_j P8_ij v8_j) * sV_max / 448 / l_i.
+
+    Pinned against ``attn_fwd_q8_blockwise`` (the per-block accumulation form):
+    the two are equal wherever no P code is subnormal, since the fold factor is
+    an exact power of two."""
     B, S, H, D = q.shape
     rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
     heads = list(range(H)) if heads is None else list(heads)
@@ -143,13 +154,55 @@ def attn_fwd_q8_sim(q, k, v, rows=None, heads=None, block: int = BLOCK):
             m = s.max(axis=1)
             p = np.exp(s - m[:, None])
             l = p.sum(axis=1)
-            sv_key = np.repeat(sv[b, h], block)[:S].astype(np.float64)        # sV of each key's block
             sv_max = float(sv[b, h].max())
-            p8 = e4m3_round(p * (E4M3_MAX * sv_key / sv_max)[None, :])
+            p8 = e4m3_round(p * (E4M3_MAX * _fold_factor(sv[b, h], S, block))[None, :])
             o[b, :, hi, :] = (p8 @ v8[b, :, h, :]) * (sv_max / E4M3_MAX) / l[:, None]
             lse[b, hi] = m + np.log(l)
     return o, lse
 
 
-__all__ = ["e4m3_round", "e4m3_bits", "quant_int8", "quant_e4m3", "attn_fwd_q8_sim",
+def attn_fwd_q8_blockwise(q, k, v, rows=None, heads=None, block: int = BLOCK):
+    """The 8-bit recipe with its cross-block accumulation written out block by block.
+
+    Wan 2.1 paper-podcast summary, section "干预与形式化" (8-bit FlashAttention:
+    per-block quantised operands, FP32 accumulation across blocks) and the kwkr.cn
+    Wan explainer, section 4.2.  For one query row i and each 64-key block t in turn:
+      scores   s_ij = (q8_i . k8_j) sQ(i) sK(t) / sqrt(D)        for j in block t
+      weights  p_ij = exp(s_ij - m_i), m_i the row's maximum over all keys
+      P codes  e4m3(448 p_ij)                 (P's own block scale: 1/448)
+      product  O_t = sum_{j in t} e4m3(448 p_ij) v8_j        (the block's 8-bit MMA)
+      add      acc += O_t * sV(t) / 448       (dequantised, accumulated across blocks)
+    and o_i = acc / l_i with l_i = sum_j p_ij (unquantised), lse_i = m_i + ln l_i.
+    No scale is folded into P here, so this form shares no step with the folded
+    simulation beyond the quantisers."""
+    B, S, H, D = q.shape
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    heads = list(range(H)) if heads is None else list(heads)
+    q8, sq = quant_int8(q, block)
+    k8, sk = quant_int8(k, block)
+    _, v8, sv = quant_e4m3(v, block)
+    nb = (S + block - 1) // block
+    o = np.empty((B, len(rows), len(heads), D))
+    lse = np.empty((B, len(heads), len(rows)))
+    for b in range(B):
+        for hi, h in enumerate(heads):
+            Qd = q8[b, rows, h, :].astype(np.float64) * sq[b, h, rows // block][:, None].astype(np.float64)
+            s_blocks = []
+            for t in range(nb):
+                kt = k8[b, t * block:(t + 1) * block, h, :].astype(np.float64) * float(sk[b, h, t])
+                s_blocks.append((Qd @ kt.T) / np.sqrt(D))
+            m = np.max([sb.max(axis=1) for sb in s_blocks], axis=0)
+            acc = np.zeros((len(rows), D))
+            l = np.zeros(len(rows))
+            for t in range(nb):
+                p = np.exp(s_blocks[t] - m[:, None])
+                l += p.sum(axis=1)
+                o_t = e4m3_round(E4M3_MAX * p) @ v8[b, t * block:(t + 1) * block, h, :]
+                acc += o_t * (float(sv[b, h, t]) / E4M3_MAX)
+            o[b, :, hi, :] = acc / l[:, None]
+            lse[b, hi] = m + np.log(l)
+    return o, lse
+
+
+__all__ = ["e4m3_round", "e4m3_bits", "quant_int8", "quant_e4m3", "attn_fwd_q8_sim", "attn_fwd_q8_blockwise",
            "block_absmax", "widen", "BLOCK"]

@@ -14,6 +14,13 @@ def pytest_configure(config):
 
 
 @pytest.fixture(scope="session")
+def built():
+    """Path of the C-ABI library, compiled in-tree first if missing or stale (no GPU needed)."""
+    from video_dit_full_b200 import build
+    return build.build()
+
+
+@pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
 

@@ -18,12 +18,6 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(wan_\w+)\s*\(", text)))
 
 
-@pytest.fixture(scope="module")
-def built():
-    from video_dit_full_b200 import build
-    return build.build()
-
-
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("wan_attn_fwd", "wan_attn_sync_status", "wan_attn_status_string"):

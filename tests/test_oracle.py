@@ -228,3 +228,14 @@ def test_planted_mistakes_are_caught(monkeypatch, kind):
     o, lse = oracle.attn_fwd(q, k, v)
     ob, lb = brute_fwd(q, k, v)
     assert not (np.allclose(o, ob, rtol=1e-9) and np.allclose(lse, lb, rtol=1e-9))
+
+
+def test_backward_by_head_threads_equal_direct_call():
+    # the GPU tests' threaded per-head evaluation stacks exactly what one call returns
+    from gpu_util import oracle_bwd_by_head
+    x = {n: rand((2, 70, 3, 16), 40 + i) for i, n in enumerate(("q", "k", "v", "do"))}
+    k_rows, q_rows = [0, 5, 69], [1, 68]
+    want = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], q_rows=q_rows, k_rows=k_rows, heads=[2, 0])
+    got = oracle_bwd_by_head(x, q_rows, k_rows, [2, 0], workers=2)
+    for n in ("dq", "dk", "dv", "lse", "dl"):
+        np.testing.assert_allclose(got[n], want[n], rtol=1e-12, atol=1e-14, err_msg=n)

@@ -6,9 +6,17 @@
 * int8 block quantisation against closed forms (absmax maps to +-127, zero
   block, ragged last block, block boundaries);
 * the diagnostic 8-bit simulation reduces to the dequantised V for S = 1 and
-  stays within the quantisation error budget of the exact oracle.
+  stays within the quantisation error budget of the exact oracle;
+* the simulation's folded form (each block's V scale carried inside P) against
+  the recipe written out block by block (each block's 8-bit product dequantised
+  by its own scale and accumulated across blocks): equal to rounding wherever no
+  P code is subnormal, with a ragged last block and block-scale ratios down to
+  2^-5; both reduce to the mean of the dequantised V when every score is equal;
+  planted mistakes in the fold (another block's scale, an exponent off by one)
+  break the equality.
 """
 import numpy as np
+import pytest
 import torch
 
 import oracle
@@ -93,3 +101,86 @@ def test_q8_sim_single_key_and_error_budget():
     rel = np.linalg.norm(os_ - oe) / np.linalg.norm(oe)
     assert 0.01 < rel < 0.045, rel
     assert np.abs(ls - le).max() < 0.05
+
+
+def _v_with_scaled_blocks(rng, S, H, D, factors):
+    """N(0,1) values with the 64-token block t multiplied by factors[t] (powers of two: exact)."""
+    v = rng.standard_normal((1, S, H, D)).astype(np.float32)
+    for t, f in enumerate(factors):
+        v[:, 64 * t:64 * (t + 1)] *= np.float32(f)
+    return v
+
+
+def _blockwise_case():
+    rng = np.random.default_rng(11)
+    S, H, D = 200, 2, 128                           # blocks of 64, 64, 64 and a ragged 8
+    q = (rng.standard_normal((1, S, H, D)) * 0.5).astype(np.float32)
+    k = (rng.standard_normal((1, S, H, D)) * 0.5).astype(np.float32)
+    v = _v_with_scaled_blocks(rng, S, H, D, [1.0, 2.0 ** -3, 2.0 ** -5, 0.5])
+    return q, k, v
+
+
+def test_q8_folded_form_equals_blockwise_accumulation():
+    q, k, v = _blockwise_case()
+    S = q.shape[1]
+    _, _, sv = q8.quant_e4m3(v)
+    ratios = sv / sv.max(axis=2, keepdims=True)
+    assert ratios.min() <= 2.0 ** -5 and len(np.unique(ratios)) >= 4      # the fold really shifts exponents
+    # no P code is subnormal: the smallest weight p = exp(s - m) times 448 * ratio stays >= 2^-6
+    for h in range(q.shape[2]):
+        p = oracle.softmax_matrix(q, k, 0, h)
+        pmin = (p / p.max(axis=1, keepdims=True)).min()
+        assert 448.0 * pmin * 0.9 * ratios[0, h].min() >= 2.0 ** -6
+    o_f, l_f = q8.attn_fwd_q8_sim(q, k, v)
+    o_b, l_b = q8.attn_fwd_q8_blockwise(q, k, v)
+    np.testing.assert_allclose(o_f, o_b, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l_f, l_b, rtol=0, atol=1e-12)
+    rows = np.array([0, 63, 64, 199])
+    o_r, _ = q8.attn_fwd_q8_blockwise(q, k, v, rows=rows, heads=[1])
+    np.testing.assert_allclose(o_r[:, :, 0], o_b[:, rows, 1], rtol=1e-12, atol=1e-13)
+    assert S == 200
+
+
+def test_q8_uniform_scores_reduce_to_mean_of_dequantised_v():
+    rng = np.random.default_rng(12)
+    S, H, D = 150, 2, 16
+    q = np.zeros((1, S, H, D), dtype=np.float32)
+    k = rng.standard_normal((1, S, H, D)).astype(np.float32)
+    v = _v_with_scaled_blocks(rng, S, H, D, [1.0, 0.25, 4.0])
+    _, vals, sv = q8.quant_e4m3(v)
+    deq = vals * np.repeat(sv, 64, axis=2)[:, :, :S].transpose(0, 2, 1)[:, :, :, None]
+    want = np.broadcast_to(deq.mean(axis=1, keepdims=True), (1, S, H, D))
+    for fn in (q8.attn_fwd_q8_sim, q8.attn_fwd_q8_blockwise):
+        o, lse = fn(q, k, v)
+        np.testing.assert_allclose(o, want, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(lse, np.log(S), rtol=0, atol=1e-12)
+
+
+def test_q8_forms_differ_only_by_subnormal_codes_on_peaky_scores():
+    rng = np.random.default_rng(13)
+    S, H, D = 256, 1, 128
+    q = (rng.standard_normal((1, S, H, D)) * 3).astype(np.float32)   # weights far below 2^-6 / 448
+    k = rng.standard_normal((1, S, H, D)).astype(np.float32)
+    v = _v_with_scaled_blocks(rng, S, H, D, [1.0, 2.0 ** -4, 1.0, 2.0 ** -2])
+    o_f, _ = q8.attn_fwd_q8_sim(q, k, v)
+    o_b, _ = q8.attn_fwd_q8_blockwise(q, k, v)
+    rel = np.linalg.norm(o_f - o_b) / np.linalg.norm(o_b)
+    assert 0 < rel < 1e-2, rel        # subnormal P codes round on different grids; nothing else differs
+
+
+@pytest.mark.parametrize("kind", ["neighbour_block_scale", "exponent_off_by_one", "unfolded_scale"])
+def test_q8_planted_fold_mistakes_are_caught(monkeypatch, kind):
+    good = q8._fold_factor
+
+    def bad(sv_bh, S, block):
+        f = good(sv_bh, S, block)
+        if kind == "neighbour_block_scale":        # key j takes the scale of the block before its own
+            return np.concatenate([f[:block], f[:-block]])
+        if kind == "exponent_off_by_one":          # 2^(k - kmax + 1) instead of 2^(k - kmax)
+            return np.minimum(2.0 * f, 1.0)
+        return np.ones_like(f)                     # the block scale forgotten
+    monkeypatch.setattr(q8, "_fold_factor", bad)
+    q, k, v = _blockwise_case()
+    o_f, _ = q8.attn_fwd_q8_sim(q, k, v)
+    o_b, _ = q8.attn_fwd_q8_blockwise(q, k, v)
+    assert np.linalg.norm(o_f - o_b) / np.linalg.norm(o_b) > 1e-3

@@ -51,24 +51,27 @@ def test_q8_quantisation_is_bit_exact(B, S, H):
     np.testing.assert_array_equal(v8, want_bits.transpose(0, 2, 1, 3))
 
 
-def check(x, rows=None):
+def check(x, rows=None, with_sim=True):
     o, lse, _ = run_q8(x)
     want_o, want_lse = oracle.attn_fwd(x["q"], x["k"], x["v"], rows=rows)
-    sim_o, _ = quant8.attn_fwd_q8_sim(x["q"], x["k"], x["v"], rows=rows)
+    sim_o = quant8.attn_fwd_q8_sim(x["q"], x["k"], x["v"], rows=rows)[0] if with_sim else None
     got_o = bf16_to_f64(o)
     got_lse = lse.cpu().numpy().astype(np.float64)
     if rows is not None:
         got_o, got_lse = got_o[:, rows], got_lse[:, :, rows]
     assert np.all(np.isfinite(got_o)) and np.all(np.isfinite(got_lse))
     max_abs, rel = errors(got_o, want_o)
-    _, rel_sim = errors(got_o, sim_o)
-    _, rel_recipe = errors(sim_o, want_o)
     lse_err = float(np.abs(got_lse - want_lse).max())
-    print(f"q8 O rel-frob vs exact {rel:.3e} (recipe alone {rel_recipe:.3e}, kernel vs recipe {rel_sim:.3e}) "
-          f"max-abs {max_abs:.3e} LSE {lse_err:.3e}")
+    msg = (f"q8 O rel-frob vs exact {rel:.4e} (margin to the bar {(REL_FROB - rel) / REL_FROB:+.2%}) "
+           f"max-abs {max_abs:.3e} LSE {lse_err:.3e}")
+    if sim_o is not None:
+        _, rel_sim = errors(got_o, sim_o)
+        _, rel_recipe = errors(sim_o, want_o)
+        msg += f"; recipe alone {rel_recipe:.4e}, kernel vs recipe {rel_sim:.3e}"
+        if x["q"].shape[1] <= 64:
+            assert rel_sim <= 5e-3, rel_sim
+    print(msg)
     assert rel <= REL_FROB, rel
-    if x["q"].shape[1] <= 64:
-        assert rel_sim <= 5e-3, rel_sim
     assert lse_err <= 2e-2, lse_err
 
 
@@ -81,10 +84,13 @@ def test_q8_oracle_sized_workload_full():
     check(synth.make_inputs(synth.WORKLOADS["oracle_1280"]))
 
 
-def test_q8_720p_sampled_rows():
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_q8_720p_sampled_rows(seed):
+    # four seeded draws of the 720p 8-bit workload; the fp64 simulation of the recipe (a
+    # diagnostic, minutes of CPU at this size) runs on the first only
     w = synth.WORKLOADS["q8_720p"]
-    x = synth.make_inputs(w)
-    check(x, rows=synth.sample_rows(w.S, 256))
+    x = synth.make_inputs(w, seed=seed)
+    check(x, rows=synth.sample_rows(w.S, 256, seed=seed), with_sim=(seed == 0))
 
 
 def test_q8_increasing_scores_rescale_every_block():
