@@ -113,14 +113,38 @@ def nvsmi_id(dev, local: int) -> str:
     return ids[local] if local < len(ids) else str(local)
 
 
-def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
-    """Time the fp64 oracle on `rows_per_head` query rows of every (batch, head)."""
-    import oracle
+def host_cores() -> dict:
+    """Threads the oracle's BLAS runs on, the host's CPU count and the CPUs this process may use."""
     try:
         from threadpoolctl import threadpool_info
-        cores = max(int(i.get("num_threads", 1)) for i in threadpool_info()) if threadpool_info() else 1
-    except Exception:
-        cores = os.cpu_count() or 1
+        info = threadpool_info()
+        blas = max(int(i.get("num_threads", 1)) for i in info) if info else 1
+    except Exception:  # noqa: BLE001
+        blas = os.cpu_count() or 1
+    try:
+        allowed = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        allowed = os.cpu_count() or 1
+    return {"cores": blas, "nproc": os.cpu_count() or 1, "cpus_allowed": allowed}
+
+
+def _baseline(flop, dt, sample, full_flop, cores) -> dict:
+    rate = flop / dt
+    rec = {"value": rate / 1e12, "unit": "TFLOP/s", **cores, "kind": "oracle", "sample": sample,
+           "sample_s": dt, "_flop": flop}
+    if flop >= full_flop * (1 - 1e-12):
+        rec["full_problem_s"] = dt
+    else:
+        rec["full_problem_s_extrapolated"] = full_flop / rate
+        rec["extrapolation"] = "the workload's full count of the metric's FLOPs at the sample's measured rate"
+    return rec
+
+
+def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
+    """Time the fp64 oracle on `rows_per_head` query rows of every (batch, head): a bounded
+    sample of the workload, with the full problem's time extrapolated from its rate."""
+    import oracle
+    cores = host_cores()
     if w.gemm:
         from oracle import fp8_gemm
         M, N, K = w.gemm
@@ -133,9 +157,8 @@ def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
         fp8_gemm.gemm_from_codes(xv, sx, wv, sw)
         dt = time.perf_counter() - t0
         flop = 2.0 * len(rows) * N * K
-        return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                "sample": f"{len(rows)} token rows of {w.name} (quantised) against the whole quantised "
-                          f"{N} x {K} weight, fp64 numpy/BLAS, {dt:.2f} s", "_flop": flop}
+        return _baseline(flop, dt, f"{len(rows)} token rows of {w.name} (quantised) against the whole quantised "
+                                   f"{N} x {K} weight, fp64 numpy/BLAS, {dt:.2f} s", w.fwd_flop, cores)
     if w.sparse_keep:
         from oracle import block_sparse
         if x is None:
@@ -148,19 +171,28 @@ def cpu_baseline(w, rows_per_head: int, seed: int = 0, x=None):
         block_sparse.attn_fwd_block_sparse(x["q"], x["k"], x["v"], mask, rows=rows)
         dt = time.perf_counter() - t0
         flop = float(4.0 * w.D * (mask[:, :, rows // 64, :].astype(np.float64) @ size).sum())
-        return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                "sample": f"{len(rows)} query rows x {w.B * w.H} (batch, head) pairs of {w.name} against "
-                          f"their allowed key blocks (fp64, masked dense rows), {dt:.2f} s", "_flop": flop}
+        full = float(4.0 * w.D * np.einsum("bhij,i,j->", mask.astype(np.float64), size, size))
+        return _baseline(flop, dt, f"{len(rows)} query rows x {w.B * w.H} (batch, head) pairs of {w.name} against "
+                                   f"their allowed key blocks (fp64, masked dense rows), {dt:.2f} s", full, cores)
     if x is None:
         x = synth.make_inputs(w, seed)
     rows = synth.sample_rows(w.S, rows_per_head, seed=seed)
+    full = w.fwd_flop * (3.5 if w.backward else 1.0)
+    if w.backward:
+        # the rows' forward and their dQ (scores recomputed, dP, dS K): 10 * Skv * D per row
+        t0 = time.perf_counter()
+        oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], q_rows=rows, k_rows=[])
+        dt = time.perf_counter() - t0
+        flop = 10.0 * w.B * w.H * len(rows) * w.kv_len * w.D
+        return _baseline(flop, dt, f"forward + dQ of {len(rows)} query rows x {w.B * w.H} (batch, head) pairs of "
+                                   f"{w.name} against all {w.kv_len} keys, fp64 numpy/BLAS, {dt:.2f} s", full, cores)
     t0 = time.perf_counter()
     oracle.attn_fwd(x["q"], x["k"], x["v"], rows=rows)
     dt = time.perf_counter() - t0
     flop = 4.0 * w.B * w.H * len(rows) * w.kv_len * w.D
-    return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{len(rows)} query rows x {w.B * w.H} (batch, head) pairs of {w.name} "
-                      f"against all {w.kv_len} keys, fp64 numpy/BLAS, {dt:.2f} s", "_flop": flop}
+    what = "exact (unquantised) forward" if w.q8 else "forward"
+    return _baseline(flop, dt, f"{what} of {len(rows)} query rows x {w.B * w.H} (batch, head) pairs of {w.name} "
+                               f"against all {w.kv_len} keys, fp64 numpy/BLAS, {dt:.2f} s", full, cores)
 
 
 def metric_of(w) -> str:
@@ -291,10 +323,12 @@ class Path:
         self.h2d_bytes = sum(t.numel() * t.element_size() for t in self.host_in)
         self.d2h_bytes = sum(t.numel() * t.element_size() for t in self.host_out)
 
-    def step(self, dom_events=None):
+    def step(self, dom_events=None, fwd_event=None):
         wa, (q, k, v) = self.wa, self.dev_in[:3]
         fwd = wa.cross_fwd if self.w.cross else wa.fwd
         if self.w.backward:
+            if fwd_event is not None:
+                fwd_event.record()
             fwd(q, k, v, self.o, self.lse)
             if dom_events:
                 dom_events[0].record()
@@ -576,6 +610,164 @@ def gemm_inputs(w, seed):
     return {"x": synth.make_tensor((M, K), seed, synth.STREAM_Q), "w": synth.make_tensor((N, K), seed, synth.STREAM_K)}
 
 
+# The configurations quoted beside the headline one: each gets its own record in the
+# line's "extra" object (timed on its own, with its own clocks and CPU-oracle sample).
+# Values: (timed steps, oracle query rows per (batch, head) for its cpu_baseline).
+EXTRA_WORKLOADS = {"oracle_1280": (200, 1280), "wan1.3b_480p_cfg": (20, 16),
+                   "train_480p_fwd_bwd": (8, 16), "q8_720p": (10, 16)}
+
+
+def measure_8bit_peaks(dev, n: int = 8192, reps: int = 10) -> dict:
+    """Dense 8-bit tensor throughput of this GPU through the vendor library, as the bf16 peak
+    beside it was measured: an e4m3 x e4m3 -> bf16 torch._scaled_mm and an int8 x int8 -> int32
+    torch._int_mm of n^3 (2 n^3 operations), best of `reps` launches after warm-up, CUDA events."""
+    import torch
+    out = {"shape": f"{n}x{n}x{n}", "how": f"best of {reps} launches after 3 warm-ups, CUDA events"}
+
+    def best_rate(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    try:
+        a = (torch.randn(n, n, device=dev, generator=g)).to(torch.float8_e4m3fn)
+        b = (torch.randn(n, n, device=dev, generator=g)).to(torch.float8_e4m3fn).t()   # column-major
+        one = torch.ones((), device=dev)
+        out["fp8_e4m3_tflops"] = best_rate(lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one,
+                                                                     out_dtype=torch.bfloat16))
+        del a, b
+    except Exception as e:  # noqa: BLE001 - report, do not fail the bench
+        out["fp8_e4m3_error"] = f"{type(e).__name__}: {e}"[:200]
+    try:
+        ai = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+        bi = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+        rates = {"row_major_b": best_rate(lambda: torch._int_mm(ai, bi))}
+        bt = bi.t().contiguous().t()                                                    # column-major
+        rates["col_major_b"] = best_rate(lambda: torch._int_mm(ai, bt))
+        out["int8_tops"] = max(rates.values())
+        out["int8_by_layout"] = rates
+        del ai, bi, bt
+    except Exception as e:  # noqa: BLE001
+        out["int8_error"] = f"{type(e).__name__}: {e}"[:200]
+    torch.cuda.empty_cache()
+    return out
+
+
+def peak_for(path, peaks, p8) -> tuple:
+    """(burst peak, sustained peak or None, description) for the path's dominant kernel."""
+    if path.peak_key != "fp8":
+        return peaks["bf16"], peaks["bf16_sustained"], f"{peaks['source']} bf16 dense (burst)"
+    fp8, i8 = p8.get("fp8_e4m3_tflops"), p8.get("int8_tops")
+    if isinstance(path, GemmPath):
+        if fp8:
+            return fp8, None, "measured e4m3 torch._scaled_mm 8192^3 (burst), this run"
+    elif fp8 and i8:
+        # half of the 8-bit forward's operations are int8 (Q K^T), half e4m3 (P V): time adds
+        eff = 2.0 / (1.0 / i8 + 1.0 / fp8)
+        return eff, None, ("measured, this run: 2 / (1/int8 + 1/e4m3) of torch._int_mm and "
+                           "torch._scaled_mm 8192^3 (burst); half the operations are int8 Q K^T, half e4m3 P V")
+    return (2.0 * peaks["bf16"], 2.0 * peaks["bf16_sustained"],
+            f"{peaks['source']} bf16 dense burst x 2 (nominal 8-bit : bf16 ratio; no 8-bit peak measured)")
+
+
+def time_device(path, steps, warmup, dev, wa, gpu_id, barrier=lambda: None, flush=None) -> dict:
+    """Warm-up, then `steps` steps between CUDA events on the launching stream (synchronised
+    on both sides), the dominant call timed per step, clocks sampled during the timed region.
+    `flush`: a device buffer larger than the L2, overwritten between steps (outside the
+    per-step events) when the workload's inputs would otherwise stay in the L2."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        path.step()
+    status = wa.sync_status()
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev = [(mk(), mk()) for _ in range(steps)]
+    fwd_ev = [mk() for _ in range(steps)] if isinstance(path, Path) and path.w.backward else None
+    sampler = ClockSampler(gpu_id)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    t_start, t_end = mk(), mk()
+    t_start.record(stream)
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        if fwd_ev:
+            path.step(ev[i], fwd_ev[i])
+        else:
+            path.step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier()
+    status = status or wa.sync_status()
+    return {"total_ms": t_start.elapsed_time(t_end), "dom_ms": [a.elapsed_time(b) for a, b in ev],
+            "fwd_ms": [f.elapsed_time(a) for f, (a, _) in zip(fwd_ev, ev)] if fwd_ev else None,
+            "clocks": clocks, "status": status}
+
+
+def roofline_of(path, w, t, peaks, p8) -> dict:
+    mean_ms = sum(t["dom_ms"]) / len(t["dom_ms"])
+    achieved = path.dominant_flop / (mean_ms * 1e-3) / 1e12
+    peak, sustained, src = peak_for(path, peaks, p8)
+    r = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+         "traffic": TRAFFIC.get(w.name), "peak_source": src}
+    if sustained:
+        r["frac_of_sustained"] = achieved / sustained
+    r["kernel"] = path.kernel
+    r["launch_ms"] = {"mean": mean_ms, "min": min(t["dom_ms"]), "max": max(t["dom_ms"])}
+    return r
+
+
+def extra_record(wa, name, dev, gpu_id, peaks, p8, warmup, no_cpu) -> dict:
+    """One configuration beside the headline: timed alone, with its own roofline, clocks and
+    a bounded CPU-oracle sample."""
+    import torch
+    w = synth.WORKLOADS[name]
+    steps, cpu_rows = EXTRA_WORKLOADS[name]
+    x = synth.make_inputs(w, seed=0)
+    x["seed"] = 0
+    path = make_path(wa, w, dev, x)
+    in_bytes = sum(t_.numel() * t_.element_size() for t_ in path.dev_in)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if in_bytes < 126e6 else None
+    t = time_device(path, steps, max(3, warmup), dev, wa, gpu_id, flush=flush)
+    # with an L2 flush between steps, a step's time is its own events' (the flush is outside them)
+    step_ms = sum(t["dom_ms"]) / steps if flush is not None else t["total_ms"] / steps
+    rec = {"metric": metric_of(w), "value": path.flop / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "steps": steps, "warmup": max(3, warmup), "ms_per_step": step_ms, "dtype": path.dtype,
+           "config": {**workload_config(w), "flop_per_step": path.flop}, "gpu_launches": steps * path.launches_per_step,
+           "roofline": roofline_of(path, w, t, peaks, p8), "clocks": t["clocks"], "device_status": t["status"]}
+    if t["fwd_ms"]:
+        fwd_ms = sum(t["fwd_ms"]) / len(t["fwd_ms"])
+        bwd_ms = rec["roofline"]["launch_ms"]["mean"]
+        rec["split"] = {"fwd_ms": fwd_ms, "fwd_tflops": w.fwd_flop / (fwd_ms * 1e-3) / 1e12,
+                        "bwd_ms": bwd_ms, "bwd_tflops": 2.5 * w.fwd_flop / (bwd_ms * 1e-3) / 1e12,
+                        "bwd_flop_count": "2.5 x the forward's 4*B*H*S^2*D (the pages' beta: 2x)"}
+    if w.S < 148 * 256:
+        rec["config"]["note"] = "latency-bound: fewer Q-tile CTAs than one wave of the 148 SMs"
+    rec["config"]["l2"] = ("inputs (%.1f MB) fit in the 126 MB L2: a 256 MB buffer is overwritten between "
+                           "steps, outside each step's events" % (in_bytes / 1e6) if flush is not None
+                           else "inputs (%.2f GB) exceed the 126 MB L2; no flush" % (in_bytes / 1e9))
+    del path, flush
+    torch.cuda.empty_cache()
+    if not no_cpu:
+        cb = cpu_baseline(w, cpu_rows, x=x)
+        cb.pop("_flop")
+        rec["cpu_baseline"] = cb
+    return rec
+
+
 def run_ours(args, w):
     import torch
     import video_dit_full_b200 as wa
@@ -592,38 +784,21 @@ def run_ours(args, w):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     wa.lib()
+    gpu_id = nvsmi_id(dev, local)
 
     # each rank gets its own seeded problem (seed = rank): weak scaling
     x = gemm_inputs(w, rank) if w.gemm else synth.make_inputs(w, seed=rank)
     x["seed"] = rank
     path = make_path(wa, w, dev, x)
-    stream = torch.cuda.current_stream(dev)
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
     # ------------------------ device-resident timing ------------------------
-    for _ in range(args.warmup):
-        path.step()
-    status = wa.sync_status()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    sampler = ClockSampler(nvsmi_id(dev, local))
-    barrier()
-    torch.cuda.synchronize(dev)
-    sampler.start()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for s in range(args.steps):
-        path.step(ev[s])
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    clocks = sampler.stop()
-    barrier()
-    status = status or wa.sync_status()
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
-    dom_ms = [a.elapsed_time(b) for a, b in ev]
+    t = time_device(path, args.steps, args.warmup, dev, wa, gpu_id, barrier)
+    status = t["status"]
+    total_ms = max_over_ranks(t["total_ms"], dist, dev)
     ms_per_step = total_ms / args.steps
     value = whole_job_tflops(world, path.flop, args.steps, total_ms)
 
@@ -645,16 +820,8 @@ def run_ours(args, w):
 
     if rank == 0:
         peaks = load_peaks()
-        mean_ms = sum(dom_ms) / len(dom_ms)
-        achieved = path.dominant_flop / (mean_ms * 1e-3) / 1e12
-        if path.peak_key == "fp8":
-            peak = 2.0 * peaks["bf16"]
-            peak_src = f"{peaks['source']} bf16 dense burst x 2 (nominal fp8/int8 : bf16 ratio)"
-            sustained = 2.0 * peaks["bf16_sustained"]
-        else:
-            peak, sustained = peaks["bf16"], peaks["bf16_sustained"]
-            peak_src = f"{peaks['source']} bf16 dense (burst)"
-        in_gb = sum(t.numel() * t.element_size() for t in path.dev_in) / 1e9
+        p8 = measure_8bit_peaks(dev) if world == 1 and (path.peak_key == "fp8" or not args.no_extra) else {}
+        in_gb = sum(t_.numel() * t_.element_size() for t_ in path.dev_in) / 1e9
         line = {
             "metric": metric_of(w),
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -667,20 +834,30 @@ def run_ours(args, w):
             **({"sparse": {"keep": w.sparse_keep, "union_fraction_computed": path.union_frac,
                            "dense_equivalent_tflops": whole_job_tflops(world, path.dense_flop, args.steps, total_ms)}}
                if w.sparse_keep else {}),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": TRAFFIC.get(w.name),
-                         "peak_source": peak_src, "frac_of_sustained": achieved / sustained,
-                         "kernel": path.kernel,
-                         "launch_ms": {"mean": mean_ms, "min": min(dom_ms), "max": max(dom_ms)}},
+            "roofline": roofline_of(path, w, t, peaks, p8),
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": path.h2d_bytes,
                     "d2h_bytes_per_step": path.d2h_bytes, "steps": e2e_steps,
                     "pipelined": "two buffer sets; each step's copies overlap the neighbouring steps' kernels"},
-            "clocks": clocks,
+            "clocks": t["clocks"],
             "device_status": status,
         }
+        if p8:
+            line["peaks_8bit"] = p8
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows, x=x)
             line["cpu_baseline"].pop("_flop")
+        if world == 1 and not args.no_extra:
+            del path
+            x = None
+            torch.cuda.empty_cache()
+            line["extra"] = {}
+            for name in EXTRA_WORKLOADS:
+                if name == w.name:
+                    continue
+                rec = extra_record(wa, name, dev, gpu_id, peaks, p8, args.warmup, args.no_cpu_baseline)
+                status = status or rec["device_status"]
+                line["extra"][name] = rec
+            line["device_status"] = status
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
@@ -698,6 +875,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=128, help="query rows per head timed for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="query rows per head per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other configurations' records (and the 8-bit peak measurement)")
     ap.add_argument("--S", type=int, default=None, help="override the token count (small profiling cases)")
     ap.add_argument("--H", type=int, default=None, help="override the head count (small profiling cases)")
     args = ap.parse_args()

@@ -30,6 +30,10 @@
  *     While the status word holds an error, a wait that has lasted 1 ms
  *     gives up too (healthy waits are far shorter), so that the CTAs of a
  *     call that timed out do not each spend a whole budget.
+ *   - The library looks up the device addresses of its own static device
+ *     variables (the status word; the no-alloc backward's array) once per
+ *     device and keeps them for the life of the process.  Do not keep using
+ *     it on a device after cudaDeviceReset.
  */
 #ifndef WAN_ATTN_H
 #define WAN_ATTN_H
@@ -90,8 +94,9 @@ WAN_ATTN_API size_t wan_attn_bwd_workspace_size(int B, int S, int H, int D);
  * The softmax matrix is recomputed from lse, never stored: P = exp(S/sqrt(D)
  * - lse), dS = P * (dP - D), dV = P^T dO, dK = dS^T Q / sqrt(D), dQ = dS K /
  * sqrt(D) (the non-causal backward of the cost model's beta = 8 term).
- * dQ is accumulated in fp32 in the workspace across key tiles (atomic adds),
- * so its low bits may differ between runs; dK and dV are deterministic.
+ * dQ is accumulated in fp32 in the workspace across key tiles (asynchronous
+ * bulk reduce-adds of each tile's partial, in no fixed order), so its low bits
+ * may differ between runs; dK and dV are deterministic.
  */
 WAN_ATTN_API int wan_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
                               const float* lse, void* dq, void* dk, void* dv, int B, int S, int H, int D,
@@ -305,8 +310,12 @@ WAN_ATTN_API int wan_attn_fwd_q8(const void* q, const void* k, const void* v, vo
 
 /*
  * Size of the library's own backward workspace used by wan_attn_bwd_noalloc:
- * 32 MiB, held on every GPU that loads the library until the process exits.
- * It fits B*S*H <= 65027 (token, head) rows, e.g. B=1, S=2048, H=24.
+ * 32 MiB of static device memory in the library's module.  The CUDA runtime
+ * loads that module on a device at the latest when the first
+ * wan_attn_bwd_noalloc call on that device looks the array up (earlier when
+ * lazy module loading is off); from then on the device holds the 32 MiB until
+ * the process exits.  It fits B*S*H <= 65027 (token, head) rows, e.g. B=1,
+ * S=2048, H=31.
  */
 #define WAN_ATTN_NOALLOC_WORKSPACE_BYTES (32u << 20)
 
@@ -320,9 +329,14 @@ WAN_ATTN_API int wan_attn_fwd_q8(const void* q, const void* k, const void* v, vo
  * a fixed WAN_ATTN_NOALLOC_WORKSPACE_BYTES device array inside the library.
  *   - Sizes whose wan_attn_bwd_workspace_size(B, S, H, D) exceeds that array
  *     return WAN_ATTN_ERR_WORKSPACE and enqueue nothing.
- *   - The call allocates and frees nothing.  Its first call on a device looks
- *     up the array's device address (cudaGetSymbolAddress) with that device
- *     current; make that first call before any stream capture.
+ *   - The call allocates and frees nothing itself.  Its first call on a
+ *     device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current, which can load the module and so reserve the
+ *     32 MiB (the one implicit reservation); make that first call at
+ *     start-up, before any stream capture.  The address is kept per device
+ *     for the life of the process: do not keep using the library on a device
+ *     after cudaDeviceReset (the module, and with it the array and the
+ *     library's status word, may come back at another address).
  *   - Every call on a device shares the one array.  Calls whose kernels
  *     overlap on the GPU (other streams, other host threads) race on it:
  *     order them on one stream or with events.  Each call clears what must

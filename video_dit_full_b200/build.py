@@ -52,7 +52,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
         subprocess.check_call(cmd)
     if force or not os.path.exists(OUT) or any(os.path.getmtime(o) > os.path.getmtime(OUT) for o in objs):
         tmp = OUT + f".tmp{os.getpid()}"
-        subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcuda" if False else "-lcudart_static"])
+        subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static"])
         os.replace(tmp, OUT)
     return OUT
 
