@@ -208,9 +208,9 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
 
     const bool per_tile = cross && Sq != Skv && Skv <= 1024;
     const int kv_box = per_tile ? 64 : 128;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!make_bshd_map(&tq, q, B, Sq, H, D, 128) || !make_bshd_map(&tk, k, B, Skv, H, D, kv_box) ||
-        !make_bshd_map(&tv, v, B, Skv, H, D, kv_box))
+        !make_bshd_map(&tv, v, B, Skv, H, D, kv_box) || !make_bshd_map(&to, o, B, Sq, H, D, 128))
         return WAN_ATTN_ERR_CUDA;
     FwdParams p{};
     p.o = o;
@@ -227,10 +227,10 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
         p.nqb = (Sq + 63) / 64;
         p.nkb = (Skv + 63) / 64;
         p.nctas = (Sq + 127) / 128;
-        return launch_fwd_tiles(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
-                                                                                       : WAN_ATTN_ERR_CUDA;
+        return launch_fwd_tiles(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                           : WAN_ATTN_ERR_CUDA;
     }
-    return launch_fwd(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
+    return launch_fwd(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
 }
 
 // Block-sparse forward: per 128-row Q tile (2 query blocks of 64) the list of attended key
@@ -264,9 +264,9 @@ int fwd_block_sparse_impl(const void* q, const void* k, const void* v, void* o, 
         for (size_t c = a + 1; c < 3; ++c)
             if (overlaps(outs[a], outs[c])) return WAN_ATTN_ERR_INVALID_ARG;
     }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!make_bshd_map(&tq, q, B, Sq, H, D, 128) || !make_bshd_map(&tk, k, B, Skv, H, D, 64) ||
-        !make_bshd_map(&tv, v, B, Skv, H, D, 64))
+        !make_bshd_map(&tv, v, B, Skv, H, D, 64) || !make_bshd_map(&to, o, B, Sq, H, D, 128))
         return WAN_ATTN_ERR_CUDA;
     FwdParams p{};
     p.o = o;
@@ -286,8 +286,8 @@ int fwd_block_sparse_impl(const void* q, const void* k, const void* v, void* o, 
     p.wait_budget_ns = wait_budget_ns();
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
-    return launch_fwd_tiles(tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
-                                                                                   : WAN_ATTN_ERR_CUDA;
+    return launch_fwd_tiles(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                       : WAN_ATTN_ERR_CUDA;
 }
 
 // Backward workspace: fp32 dQ accumulator [B, Sq, H, D], fp32 D_i [B, H, Sq] and, for the
@@ -449,9 +449,9 @@ int wan_attn_fwd_q8(const void* q, const void* k, const void* v, void* o, float*
     qp.S = S;
     qp.H = H;
     qp.nblk = nblk;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!make_bh_s_d8_map(&tq, qp.q8, B * H, S, 128) || !make_bh_s_d8_map(&tk, qp.k8, B * H, S, 64) ||
-        !make_bh_s_d8_map(&tv, qp.v8, B * H, S, 64))
+        !make_bh_s_d8_map(&tv, qp.v8, B * H, S, 64) || !make_bshd_map(&to, o, B, S, H, D, 128))
         return WAN_ATTN_ERR_CUDA;
     Q8AttnParams p;
     p.o = o;
@@ -467,7 +467,8 @@ int wan_attn_fwd_q8(const void* q, const void* k, const void* v, void* o, float*
     p.wait_budget_ns = wait_budget_ns();
     p.status = device_status_word();
     if (!p.status) return WAN_ATTN_ERR_CUDA;
-    return launch_q8(qp, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK : WAN_ATTN_ERR_CUDA;
+    return launch_q8(qp, tq, tk, tv, to, p, static_cast<cudaStream_t>(stream)) == 0 ? WAN_ATTN_OK
+                                                                                    : WAN_ATTN_ERR_CUDA;
 }
 
 int wan_attn_cp_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,

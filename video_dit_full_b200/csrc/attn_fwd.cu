@@ -17,7 +17,8 @@
 //   warps 0-3   softmax of Q tile 0, warps 4-7 of Q tile 1: one row per thread,
 //               online max / sum in fp32 with exp2, the running max only moved
 //               when it rises by more than 2^8 (O rescaled in TMEM then), P
-//               written back to TMEM as bf16; epilogue O / l -> bf16, LSE.
+//               written back to TMEM as bf16; epilogue O / l -> bf16 through the
+//               tile's Q buffer and two TMA stores, LSE.
 // The two Q tiles ping-pong: while one softmax group works on its S, the
 // tensor core runs the other tile's P V and Q K^T.
 #include <cuda.h>
@@ -73,7 +74,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 
 __global__ void __launch_bounds__(NTHREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
+                const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo, const FwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -274,29 +275,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             mbar_arrive(bar(P_FULL + t));
         }
         if (ok) ok = wait_warp(bar(O_FINAL + t), 0, wc);
+        // O / l as bf16 goes through this tile's Q buffer, which every MMA that read it has
+        // finished with (the tile's last Q K^T precedes its last P V, whose completion O_FINAL
+        // signals): each thread writes its row in the tensor map's 128-byte-swizzled layout, then
+        // one thread stores the tile with two TMA stores (rows past S are not written).
+        const uint32_t stage = sQ + t * TILE_BYTES;
         if (ok) {
             tc_fence_after();
             const float inv_l = 1.f / l;
-            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                  ((static_cast<size_t>(b) * p.S + row) * p.H + h) * HD;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                uint32_t o[32];
-                tmem_ld32(tO + q * 32, o);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t o[64];
+                tmem_ld32(tO + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                tmem_ld32(tO + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
                 tmem_wait_ld();
-                uint4 pk[4];
-                uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+                uint32_t w[32];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pw[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-                if (row < p.S) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = pk[e];
-                }
+                for (int e = 0; e < 32; ++e)
+                    w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                st_row_sw128(stage + half * HALF_BYTES, r, w);
             }
+            fence_proxy_async_smem();
             if (row < p.S)
                 p.lse[(static_cast<size_t>(b) * p.H + h) * p.S + row] = (m_ref + log2f(l)) * 0.69314718055994531f;
+        }
+        named_bar_sync(1 + t, BM);                // every warp of the group, whatever its state
+        if (r == 0 && ok && !*abort_flag) {
+            tma_store_4d(&tmo, stage, 0, h, q0 + t * BM, b);
+            tma_store_4d(&tmo, stage + HALF_BYTES, 64, h, q0 + t * BM, b);
+            bulk_commit_group();
+            bulk_wait_read_all();                 // the buffer stays valid until the copies have read it
         }
     }
 
@@ -308,11 +316,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
 
 }  // namespace fwd
 
-int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-               cudaStream_t stream) {
+int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+               const FwdParams& p, cudaStream_t stream) {
     if (configure_smem(reinterpret_cast<const void*>(fwd::attn_fwd_kernel), fwd::SMEM_BYTES) != 0) return -1;
     const dim3 grid((p.S + fwd::NQ * fwd::BM - 1) / (fwd::NQ * fwd::BM), p.H, p.B);
-    fwd::attn_fwd_kernel<<<grid, fwd::NTHREADS, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    fwd::attn_fwd_kernel<<<grid, fwd::NTHREADS, fwd::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

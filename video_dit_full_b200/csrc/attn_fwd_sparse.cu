@@ -25,8 +25,9 @@
 //                      block, which either attends the step's key block (keys past Skv
 //                      masked) or gets P = 0 for it; online max and sum in fp32 with exp2,
 //                      the running max moved only when it rises by more than 2^8 (O rescaled
-//                      in TMEM then); epilogue O / l -> bf16, LSE.  A row that attends
-//                      nothing gets O = 0 and LSE = -inf.
+//                      in TMEM then); epilogue O / l -> bf16 through the Q buffer and two
+//                      TMA stores, LSE.  A row that attends nothing gets O = 0 and
+//                      LSE = -inf.
 #include <cuda.h>
 
 #include "sm100_ptx.cuh"
@@ -81,7 +82,8 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 
 __global__ void __launch_bounds__(NTHREADS, 2)
 attn_fwd_sparse_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                       const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
+                       const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                       const FwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -295,38 +297,45 @@ attn_fwd_sparse_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_con
             if (k + 1 < n) lim_next = keep_of(k + 1);
         }
         if (ok && n > 0) ok = wait_warp(bar(O_FINAL), 0, wc);
+        // O / l as bf16 goes through the Q buffer, which every MMA that read it has finished
+        // with (the last Q K^T precedes the last P V, whose completion O_FINAL signals; with no
+        // key block nothing was loaded into it): each thread writes its row in the tensor map's
+        // 128-byte-swizzled layout, then one thread stores the tile with two TMA stores (rows
+        // past S are not written).
         if (ok) {
             tc_fence_after();
             // a row with no allowed key (l = 0, or no key block at all) gets O = 0, LSE = -inf
             const bool empty = !(l > 0.f);
             const float inv_l = empty ? 0.f : 1.f / l;
-            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                  ((static_cast<size_t>(b) * p.S + row) * p.H + h) * HD;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                uint4 pk4[4];
-                uint32_t* pw = reinterpret_cast<uint32_t*>(pk4);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t w[32];
                 if (n > 0) {                               // TMEM O is written only if a step ran
-                    uint32_t o[32];
-                    tmem_ld32(tO + q * 32, o);
+                    uint32_t o[64];
+                    tmem_ld32(tO + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                    tmem_ld32(tO + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pw[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                    for (int e = 0; e < 32; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
                 }
                 if (empty) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pw[e] = 0u;
+                    for (int e = 0; e < 32; ++e) w[e] = 0u;
                 }
-                if (row < p.S) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = pk4[e];
-                }
+                st_row_sw128(sQ + half * Q_HALF, r, w);
             }
+            fence_proxy_async_smem();
             if (row < p.S)
                 p.lse[(static_cast<size_t>(b) * p.H + h) * p.S + row] =
                     empty ? -INFINITY : (m_ref + log2f(l)) * 0.69314718055994531f;
+        }
+        named_bar_sync(1, BM);                        // every softmax warp, whatever its state
+        if (r == 0 && ok && !*abort_flag) {
+            tma_store_4d(&tmo, sQ, 0, h, q0, b);
+            tma_store_4d(&tmo, sQ + Q_HALF, 64, h, q0, b);
+            bulk_commit_group();
+            bulk_wait_read_all();                     // the buffer stays valid until the copies have read it
         }
     }
 
@@ -366,8 +375,8 @@ __global__ void __launch_bounds__(256) sparse_tile_lists_kernel(const uint8_t* _
 
 }  // namespace sparse
 
-int launch_fwd_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64, const FwdParams& p,
-                     cudaStream_t stream) {
+int launch_fwd_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64, const CUtensorMap& to,
+                     const FwdParams& p, cudaStream_t stream) {
     if (p.kv_list) {
         int sms = 148, dev = 0;
         if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -380,7 +389,7 @@ int launch_fwd_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUten
     if (configure_smem(reinterpret_cast<const void*>(sparse::attn_fwd_sparse_kernel), sparse::SMEM_BYTES) != 0)
         return -1;
     const dim3 grid(p.nctas, p.H, p.B);
-    sparse::attn_fwd_sparse_kernel<<<grid, sparse::NTHREADS, sparse::SMEM_BYTES, stream>>>(tq, tk64, tv64, p);
+    sparse::attn_fwd_sparse_kernel<<<grid, sparse::NTHREADS, sparse::SMEM_BYTES, stream>>>(tq, tk64, tv64, to, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

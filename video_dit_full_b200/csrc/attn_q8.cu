@@ -192,7 +192,8 @@ __device__ __forceinline__ void issue_pv8(uint32_t d_tmem, uint32_t p_tmem, uint
 
 __global__ void __launch_bounds__(NTHREADS, 1)
 q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-               const __grid_constant__ CUtensorMap tmv, const Q8AttnParams p) {
+               const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+               const Q8AttnParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -435,29 +436,37 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
             sv_cur = sv_next;
         }
         if (ok) ok = wait_warp(bar(O_FINAL + t), 0, wc);
+        // O goes out through the K/V ring, free once both tiles' last P V have completed (every
+        // block was consumed by both tiles' MMAs and nothing more is loaded): tile t's bf16 O in
+        // the ring's 32 KB half t, each thread writing its row in the tensor map's 128-byte-swizzled
+        // layout, then one thread stores the tile with two TMA stores (rows past S are not written).
+        if (ok && 1 - t < nq) ok = wait_warp(bar(O_FINAL + 1 - t), 0, wc);
+        const uint32_t stage = sK + static_cast<uint32_t>(t) * (2 * TQ8);
         if (ok) {
             tc_fence_after();
             // O = (sum over blocks of P8 V8) * sV_max / P_SCALE / l
             const float mul = sv_max / (P_SCALE * l);
-            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                  ((static_cast<size_t>(b) * S + row) * p.H + h) * HD;
 #pragma unroll 1
-            for (int q = 0; q < 4; ++q) {
-                uint32_t o[32];
-                tmem_ld32(tO + q * 32, o);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t o[64];
+                tmem_ld32(tO + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                tmem_ld32(tO + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
                 tmem_wait_ld();
-                uint4 pk4[4];
-                uint32_t* pw = reinterpret_cast<uint32_t*>(pk4);
+                uint32_t w[32];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pw[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
-                if (row < S) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = pk4[e];
-                }
+                for (int e = 0; e < 32; ++e)
+                    w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * mul, __uint_as_float(o[2 * e + 1]) * mul);
+                st_row_sw128(stage + half * TQ8, r, w);
             }
+            fence_proxy_async_smem();
             if (row < S) p.lse[static_cast<size_t>(bh) * S + row] = (m_ref + log2f(l)) * 0.69314718055994531f;
+        }
+        named_bar_sync(1 + t, BM);                // every warp of the group, whatever its state
+        if (r == 0 && ok && !*abort_flag) {
+            tma_store_4d(&tmo, stage, 0, h, q0 + t * BM, b);
+            tma_store_4d(&tmo, stage + TQ8, 64, h, q0 + t * BM, b);
+            bulk_commit_group();
+            bulk_wait_read_all();                 // the ring stays valid until the copies have read it
         }
     }
 
@@ -470,13 +479,13 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
 }  // namespace q8
 
 int launch_q8(const Q8QuantParams& qp, const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv8,
-              const Q8AttnParams& p, cudaStream_t stream) {
+              const CUtensorMap& to, const Q8AttnParams& p, cudaStream_t stream) {
     const long long nq = 3ll * qp.nblk * qp.B * qp.H;
     q8::q8_quantize_kernel<<<static_cast<unsigned>(nq), 256, 0, stream>>>(qp);
     if (cudaGetLastError() != cudaSuccess) return -1;
     if (configure_smem(reinterpret_cast<const void*>(q8::q8_attn_kernel), q8::SMEM_BYTES) != 0) return -1;
     const dim3 grid((p.S + q8::NQ * q8::BM - 1) / (q8::NQ * q8::BM), p.H, p.B);
-    q8::q8_attn_kernel<<<grid, q8::NTHREADS, q8::SMEM_BYTES, stream>>>(tq8, tk8, tv8, p);
+    q8::q8_attn_kernel<<<grid, q8::NTHREADS, q8::SMEM_BYTES, stream>>>(tq8, tk8, tv8, to, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -183,6 +183,40 @@ __device__ __forceinline__ void tma_reduce_add_4d(const void* tmap, uint32_t src
         "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
+// 4-D tiled store shared -> global, tracked by the issuing thread's bulk async-group.  Parts of
+// the box outside the tensor (rows past S) are not written.  The coordinates must be >= 0.
+__device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group"
+        " [%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+// Make this thread's ordinary shared-memory writes visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Barrier among `nthreads` threads (a multiple of 32) of the CTA on hardware barrier `id` (1-15).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// 16-byte shared-memory store.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+// Address of 16-byte chunk `c` (0-7) of row `r` in a [rows][128 bytes] tile at `tile` (1024-byte
+// aligned) laid out with the 128-byte swizzle that TMA uses: the chunk index is XORed with r % 8.
+__device__ __forceinline__ uint32_t sw128_chunk(uint32_t tile, int r, int c) {
+    return tile + static_cast<uint32_t>(r) * 128u + (static_cast<uint32_t>((c ^ r) & 7) << 4);
+}
+
+// A row's 64 bf16 (32 packed words) into its 128-byte row of a swizzled tile.
+__device__ __forceinline__ void st_row_sw128(uint32_t tile, int r, const uint32_t (&w)[32]) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) st_shared_v4(sw128_chunk(tile, r, c), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+}
+
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the shared-memory sources of every committed bulk group have been read.
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

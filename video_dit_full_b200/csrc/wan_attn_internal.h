@@ -77,14 +77,15 @@ unsigned long long wait_budget_ns();
 // Sets the dynamic shared-memory limit of a kernel once per device.  0 on success.
 int configure_smem(const void* kernel, int bytes);
 
-int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
-               cudaStream_t stream);
+// `to`: a map over O with the layout and box of tq (the epilogue TMA-stores O through it).
+int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+               const FwdParams& p, cudaStream_t stream);
 // Forward with one CTA per 128-row Q tile (p.nctas = the number of Q tiles), 64-key steps; tk64 /
 // tv64 are K / V maps with 64-token boxes.  Block-sparse (p.kv_list set): builds each tile's
 // key-block list in p.kv_list / p.kv_count (device workspace) from p.mask, then runs the kernel
 // over the lists.  p.kv_list null: every key block, no mask.
-int launch_fwd_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64, const FwdParams& p,
-                     cudaStream_t stream);
+int launch_fwd_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64, const CUtensorMap& to,
+                     const FwdParams& p, cudaStream_t stream);
 
 // Chooses p.nsplit (1 unless allow_split and the key tiles alone fill too few waves of the
 // GPU), then launches the backward's kernels.  tdk / tdv (fp32 accumulators, as tdq) are only
@@ -106,7 +107,8 @@ int launch_fp8_quant_tensor(const void* w, void* codes, float* scale2, long long
 int launch_fp8_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tb_half, const Fp8GemmParams& p,
                     cudaStream_t stream);
 
+// `to`: a map over the bf16 O [B, S, H, D] with 128-token boxes (the epilogue TMA-stores O through it).
 int launch_q8(const Q8QuantParams& qp, const CUtensorMap& tq8, const CUtensorMap& tk8, const CUtensorMap& tv8,
-              const Q8AttnParams& p, cudaStream_t stream);
+              const CUtensorMap& to, const Q8AttnParams& p, cudaStream_t stream);
 
 }  // namespace wan
