@@ -50,27 +50,11 @@ constexpr int SMEM_BYTES = SMEM_USED + 1024;   // slack for 1024-byte alignment 
 constexpr int NTHREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;            // S0 S1 O0 O1, 128 columns each
 constexpr float RESCALE_THRESHOLD = 8.0f;      // log2 units: keep a stale max while p <= 2^8
+#ifndef WAN_FWD_POLY_PAIRS
+#define WAN_FWD_POLY_PAIRS 0          // of every 8 pairs of exponentials, this many use exp2_poly3_x2
+#endif
+constexpr int FWD_POLY_PAIRS = WAN_FWD_POLY_PAIRS;
 
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem, uint32_t idesc) {
-    // K = 128 = 8 steps of 16; steps 0-3 in the first 64-column half, 4-7 in the second.
-#pragma unroll
-    for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-        mma_f16_ss(d_tmem, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024), idesc,
-                   kk > 0 ? 1u : 0u);
-    }
-}
-
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc,
-                                         bool accumulate) {
-    // A = P (128 x 128 bf16 in TMEM, 2 per column), B = V stored [key][d] (MN-major):
-    // 16 keys per step = 2048 bytes; the two 64-wide halves of d are 16 KB apart (LBO).
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk) {
-        mma_f16_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(v_smem + kk * 2048, HALF_BYTES, 1024), idesc,
-                   (accumulate || kk > 0) ? 1u : 0u);
-    }
-}
 
 __global__ void __launch_bounds__(NTHREADS, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -161,13 +145,30 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         if (lane == 0) {
             const uint32_t idesc_qk = make_idesc(1, 1, 1, 0, 0, BM, BN);
             const uint32_t idesc_pv = make_idesc(1, 1, 1, 0, 1, BM, HD);
+            // descriptor halves: the low half carries the address (16-byte units), the high half
+            // is one constant per operand kind.  Q K^T: 8 steps of K = 16 over the two 64-wide
+            // halves of d (Q and K both K-major); P V: 8 steps of 16 keys, P from TMEM, V [key][d]
+            // MN-major with its halves of d 16 KB apart (LBO).
+            const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024), dk0 = sdesc_sw128(sK, 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(sV, HALF_BYTES, 1024);
+            const uint32_t hi_qk = static_cast<uint32_t>(dq0 >> 32), hi_pv = static_cast<uint32_t>(dv0 >> 32);
+            const uint32_t q_lo = static_cast<uint32_t>(dq0), k_lo = static_cast<uint32_t>(dk0);
+            const uint32_t v_lo = static_cast<uint32_t>(dv0);
+            constexpr uint32_t TILE16 = TILE_BYTES >> 4;
+            auto issue_qk = [&](int t_, int s_) {
+                mma8_f16_ss<HALF_BYTES / 16>(tmem + t_ * BN, q_lo + t_ * TILE16, k_lo + s_ * TILE16, hi_qk, idesc_qk, 0u);
+            };
+            auto issue_pv = [&](int t_, int s_, bool acc) {
+                mma8_f16_ts<2048 / 16>(tmem + 256 + t_ * HD, tmem + t_ * BN, v_lo + s_ * TILE16, hi_pv, idesc_pv,
+                                       acc ? 1u : 0u);
+            };
             bool ok = true;
             for (int t = 0; t < nq && ok; ++t) ok = wait_thread(bar(Q_FULL + t), 0, wc);
             if (ok) ok = wait_thread(bar(K_FULL + 0), 0, wc);
             if (ok) {
                 tc_fence_after();
                 for (int t = 0; t < nq; ++t) {
-                    issue_qk(tmem + t * BN, sQ + t * TILE_BYTES, sK, idesc_qk);
+                    issue_qk(t, 0);
                     mma_commit(bar(S_FULL + t));
                 }
                 mma_commit(bar(K_EMPTY + 0));
@@ -180,7 +181,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     ok = wait_thread(bar(P_FULL + t), j & 1, wc);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_pv(tmem + 256 + t * HD, tmem + t * BN, sV + s * TILE_BYTES, idesc_pv, j > 0);
+                    issue_pv(t, s, j > 0);
                     if (j + 1 == nkv) mma_commit(bar(O_FINAL + t));
                     if (j + 1 < nkv) {
                         if (t == 0) {
@@ -188,7 +189,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                             if (!ok) break;
                             tc_fence_after();
                         }
-                        issue_qk(tmem + t * BN, sQ + t * TILE_BYTES, sK + s1 * TILE_BYTES, idesc_qk);
+                        issue_qk(t, s1);
                         mma_commit(bar(S_FULL + t));
                     }
                 }
@@ -244,20 +245,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 m_ref = m_cand;
                 moved = true;
             }
-            const float neg = -m_ref;
-            float sum = 0.f;
+            // P = 2^(s c - m) in packed pairs, the row sum in four independent packed accumulators.
+            // Of every 8 pairs FWD_POLY_PAIRS come from the degree-3 polynomial on the FMA pipe and
+            // the rest from the MUFU (none by default: the polynomial's extra instructions slow the
+            // MMA issuer that shares a sub-partition with the softmax warps more than they save).
+            const float2 c2 = make_float2(c, c), n2 = make_float2(-m_ref, -m_ref);
+            float2 acc[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) acc[a] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
-                    const float p0 = ex2_approx(fmaf(s[half * 64 + 2 * q], c, neg));
-                    const float p1 = ex2_approx(fmaf(s[half * 64 + 2 * q + 1], c, neg));
-                    sum += p0 + p1;
-                    pk[q] = pack_bf16x2(p0, p1);
+                    const float2 x = ffma2(make_float2(s[half * 64 + 2 * q], s[half * 64 + 2 * q + 1]), c2, n2);
+                    float2 e;
+                    if ((q & 7) < FWD_POLY_PAIRS)
+                        e = exp2_poly3_x2(x);
+                    else
+                        e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    acc[q & 3] = fadd2(acc[q & 3], e);
+                    pk[q] = pack_bf16x2(e.x, e.y);
                 }
                 tmem_st32(tS + half * 32, pk);
             }
+            const float2 acc2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+            const float sum = acc2.x + acc2.y;
             l = l * alpha + sum;
             if (j > 0 && __any_sync(0xffffffffu, moved)) {
 #pragma unroll 1

@@ -384,6 +384,66 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint
 }
 
 // Arrive once on `bar` when every tcgen05 op this thread issued before has completed.
+// The 8 MMAs of a K = 128 contraction (K = 16 each) in one asm block, A and B from shared memory
+// in two 64-wide, 128-byte-swizzled halves of K that lie `half16` * 16 bytes apart: step k reads
+// at (k / 4) * half16 + (k % 4) * 2 (in 16-byte units) past the base descriptors, whose low
+// halves are a_lo / b_lo and whose high half is `hi`.  The first MMA overwrites D unless
+// `accumulate`; the others accumulate.
+template <uint32_t half16>
+__device__ __forceinline__ void mma8_f16_ss(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t.reg .b32 x, y;\n\t.reg .b64 a, b;\n\t"
+        "setp.ne.b32 p0, %5, 0;\n\tsetp.eq.b32 p1, %4, %4;\n\t"
+        "mov.b64 a, {%1, %3};\n\tmov.b64 b, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p0;\n\t"
+        "add.u32 x, %1, 2;\n\tadd.u32 y, %2, 2;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, 4;\n\tadd.u32 y, %2, 4;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, 6;\n\tadd.u32 y, %2, 6;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, %6;\n\tadd.u32 y, %2, %6;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, %7;\n\tadd.u32 y, %2, %7;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, %8;\n\tadd.u32 y, %2, %8;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, %9;\n\tadd.u32 y, %2, %9;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t}" ::"r"(d),
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "n"(half16), "n"(half16 + 2),
+        "n"(half16 + 4), "n"(half16 + 6)
+        : "memory");
+}
+// The 8 MMAs of a K = 128 contraction with A from TMEM (a_tmem + 8 k: bf16 pairs, 16 elements
+// of K per 8 columns) and B from shared memory, step k at k * step16 (16-byte units) past the
+// base descriptor (low half b_lo, high half hi).
+template <uint32_t step16>
+__device__ __forceinline__ void mma8_f16_ts(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t hi, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t.reg .b32 x, t;\n\t.reg .b64 b;\n\t"
+        "setp.ne.b32 p0, %5, 0;\n\tsetp.eq.b32 p1, %4, %4;\n\t"
+        "mov.b64 b, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %4, p0;\n\t"
+        "add.u32 x, %2, %6;\n\tadd.u32 t, %1, 8;\n\tmov.b64 b, {x, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
+        "add.u32 x, %2, %7;\n\tadd.u32 t, %1, 16;\n\tmov.b64 b, {x, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
+        "add.u32 x, %2, %8;\n\tadd.u32 t, %1, 24;\n\tmov.b64 b, {x, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
+        "add.u32 x, %2, %9;\n\tadd.u32 t, %1, 32;\n\tmov.b64 b, {x, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
+        "add.u32 x, %2, %10;\n\tadd.u32 t, %1, 40;\n\tmov.b64 b, {x, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
+        "add.u32 x, %2, %11;\n\tadd.u32 t, %1, 48;\n\tmov.b64 b, {x, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
+        "add.u32 x, %2, %12;\n\tadd.u32 t, %1, 56;\n\tmov.b64 b, {x, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t}" ::"r"(d),
+        "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "n"(step16), "n"(2 * step16),
+        "n"(3 * step16), "n"(4 * step16), "n"(5 * step16), "n"(6 * step16), "n"(7 * step16)
+        : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
@@ -453,6 +513,21 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
+}
+
+// exp2_poly3 for a pair in packed arithmetic: the same clamp, range split, coefficients and
+// exponent-field add per element, so each result equals exp2_poly3 of its input.
+__device__ __forceinline__ float2 exp2_poly3_x2(float2 x) {
+    x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+    const float2 magic = make_float2(12582912.f, 12582912.f);
+    const float2 j = fadd2(x, magic);                       // n in the low mantissa bits
+    const float2 f = fsub2(x, fsub2(j, magic));             // exact: x - n
+    float2 p = ffma2(make_float2(0.05517149344086647f, 0.05517149344086647f), f,
+                     make_float2(0.24261093139648438f, 0.24261093139648438f));
+    p = ffma2(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+    p = ffma2(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
 }
 
 // 2^x for a pair, for results that are rounded to e4m3 next (3 mantissa bits): the same
