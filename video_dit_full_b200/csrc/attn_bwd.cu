@@ -78,33 +78,27 @@ __device__ __forceinline__ void fence_async_smem() {
 }
 
 // 8 MMAs of K = 16 over a [128 rows][128 cols] bf16 tile pair, both K-major (K = the 128 columns).
-__device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, uint32_t idesc,
-                                           bool accumulate) {
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-        mma_f16_ss(d_tmem, sdesc_sw128(a_smem + off, 16, 1024), sdesc_sw128(b_smem + off, 16, 1024), idesc,
-                   (accumulate || kk > 0) ? 1u : 0u);
-    }
+// Shared-memory operands are given as their descriptors' low halves (lo_of: address and leading
+// offset), `hi` the common high half.
+__device__ __forceinline__ uint32_t lo_kmajor(uint32_t smem) { return sdesc_lo(smem, 16); }
+__device__ __forceinline__ uint32_t lo_mnmajor(uint32_t smem) { return sdesc_lo(smem, HALF_BYTES); }
+__device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, uint32_t hi,
+                                           uint32_t idesc, bool accumulate) {
+    mma8_f16_ss<HALF_BYTES / 16, 2>(d_tmem, lo_kmajor(a_smem), lo_kmajor(b_smem), hi, idesc, accumulate ? 1u : 0u);
 }
 
 // A in TMEM (bf16, 128 x 128), B MN-major in shared memory: K = the 128 rows of the B tile.
 // A's columns for K = 0-63 start at a_tmem, those for K = 64-127 at a_tmem + 64 (each half of
 // the row is written by its own thread into the TMEM columns it has just read).
-__device__ __forceinline__ void mma_ts_bmn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, uint32_t idesc,
-                                           bool accumulate) {
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-        mma_f16_ts(d_tmem, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8, sdesc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024),
-                   idesc, (accumulate || kk > 0) ? 1u : 0u);
+__device__ __forceinline__ void mma_ts_bmn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, uint32_t hi,
+                                           uint32_t idesc, bool accumulate) {
+    mma8_f16_ts<64, 512, 128>(d_tmem, a_tmem, lo_mnmajor(b_smem), hi, idesc, accumulate ? 1u : 0u);
 }
 
 // A and B both MN-major in shared memory, K = the 128 rows of both tiles.
-__device__ __forceinline__ void mma_ss_mn(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, uint32_t idesc) {
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-        mma_f16_ss(d_tmem, sdesc_sw128(a_smem + kk * 2048, HALF_BYTES, 1024),
-                   sdesc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc, kk > 0 ? 1u : 0u);
+__device__ __forceinline__ void mma_ss_mn(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, uint32_t hi,
+                                          uint32_t idesc) {
+    mma8_f16_ss<512, 128>(d_tmem, lo_mnmajor(a_smem), lo_mnmajor(b_smem), hi, idesc, 0u);
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -208,13 +202,14 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             const uint32_t id_kk = make_idesc(1, 1, 1, 0, 0, BM, BM);   // both K-major
             const uint32_t id_tb = make_idesc(1, 1, 1, 0, 1, BM, HD);   // A in TMEM, B MN-major
             const uint32_t id_mm = make_idesc(1, 1, 1, 1, 1, HD, BM);   // both MN-major
+            const uint32_t hi = sdesc_hi();
             bool ok = wait_thread(bar(KV_FULL), 0, wc);
             if (ok) ok = wait_thread(bar(QDO_FULL + 0), 0, wc);
             if (ok) {
                 tc_fence_after();
-                mma_kmajor(tmem + T_S, sK, sQ(0), id_kk, false);      // S^T = K Q^T of the first tile
+                mma_kmajor(tmem + T_S, sK, sQ(0), hi, id_kk, false);      // S^T = K Q^T of the first tile
                 mma_commit(bar(S_FULL));
-                mma_kmajor(tmem + T_DP, sV, sDO(0), id_kk, false);    // dP^T = V dO^T
+                mma_kmajor(tmem + T_DP, sV, sDO(0), hi, id_kk, false);    // dP^T = V dO^T
                 mma_commit(bar(DP_FULL));
             }
             for (int i = 0; i < nq && ok; ++i) {
@@ -223,17 +218,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 ok = wait_thread(bar(P_READY), i & 1, wc);
                 if (!ok) break;
                 tc_fence_after();
-                mma_ts_bmn(tmem + T_DV, tmem + T_S, do_s, id_tb, i > 0);   // dV += P^T dO
+                mma_ts_bmn(tmem + T_DV, tmem + T_S, do_s, hi, id_tb, i > 0);   // dV += P^T dO
                 mma_commit(bar(DV_DONE));
                 ok = wait_thread(bar(DS_READY), i & 1, wc);
                 if (!ok) break;
                 tc_fence_after();
-                mma_ts_bmn(tmem + T_DK, tmem + T_DP, q_s, id_tb, i > 0);   // dK += dS^T Q
+                mma_ts_bmn(tmem + T_DK, tmem + T_DP, q_s, hi, id_tb, i > 0);   // dK += dS^T Q
                 ok = wait_thread(bar(DS_SMEM), i & 1, wc);
                 if (!ok) break;
                 // dQ^T = K^T dS^T (dS^T in dO's buffer) into dP^T's columns, which the dK MMA just
                 // read: S^T's columns are free for the next tile at once
-                mma_ss_mn(tmem + T_DP, sK, do_s, id_mm);
+                mma_ss_mn(tmem + T_DP, sK, do_s, hi, id_mm);
                 mma_commit(bar(DQ_FULL));
                 mma_commit(bar(QDO_EMPTY + s));
                 if (i + 1 < nq) {
@@ -243,12 +238,12 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     ok = wait_thread(bar(QDO_FULL + s1), ((i + 1) >> 1) & 1, wc);
                     if (!ok) break;
                     tc_fence_after();
-                    mma_kmajor(tmem + T_S, sK, sQ(s1), id_kk, false);
+                    mma_kmajor(tmem + T_S, sK, sQ(s1), hi, id_kk, false);
                     mma_commit(bar(S_FULL));
                     ok = wait_thread(bar(DQ_DRAINED), i & 1, wc);
                     if (!ok) break;
                     tc_fence_after();
-                    mma_kmajor(tmem + T_DP, sV, sDO(s1), id_kk, false);
+                    mma_kmajor(tmem + T_DP, sV, sDO(s1), hi, id_kk, false);
                     mma_commit(bar(DP_FULL));
                 }
             }

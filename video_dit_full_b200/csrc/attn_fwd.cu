@@ -145,22 +145,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         if (lane == 0) {
             const uint32_t idesc_qk = make_idesc(1, 1, 1, 0, 0, BM, BN);
             const uint32_t idesc_pv = make_idesc(1, 1, 1, 0, 1, BM, HD);
-            // descriptor halves: the low half carries the address (16-byte units), the high half
-            // is one constant per operand kind.  Q K^T: 8 steps of K = 16 over the two 64-wide
-            // halves of d (Q and K both K-major); P V: 8 steps of 16 keys, P from TMEM, V [key][d]
-            // MN-major with its halves of d 16 KB apart (LBO).
-            const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024), dk0 = sdesc_sw128(sK, 16, 1024);
-            const uint64_t dv0 = sdesc_sw128(sV, HALF_BYTES, 1024);
-            const uint32_t hi_qk = static_cast<uint32_t>(dq0 >> 32), hi_pv = static_cast<uint32_t>(dv0 >> 32);
-            const uint32_t q_lo = static_cast<uint32_t>(dq0), k_lo = static_cast<uint32_t>(dk0);
-            const uint32_t v_lo = static_cast<uint32_t>(dv0);
+            // descriptor halves built once: the low half carries the address (16-byte units) and
+            // the leading offset, the high half is common.  Q K^T: 8 steps of K = 16 over the two
+            // 64-wide halves of d (Q and K K-major); P V: 8 steps of 16 keys, P from TMEM, V
+            // [key][d] MN-major with its halves of d 16 KB apart (LBO).
+            const uint32_t hi = sdesc_hi();
+            const uint32_t q_lo = sdesc_lo(sQ, 16), k_lo = sdesc_lo(sK, 16), v_lo = sdesc_lo(sV, HALF_BYTES);
             constexpr uint32_t TILE16 = TILE_BYTES >> 4;
             auto issue_qk = [&](int t_, int s_) {
-                mma8_f16_ss<HALF_BYTES / 16>(tmem + t_ * BN, q_lo + t_ * TILE16, k_lo + s_ * TILE16, hi_qk, idesc_qk, 0u);
+                mma8_f16_ss<HALF_BYTES / 16, 2>(tmem + t_ * BN, q_lo + t_ * TILE16, k_lo + s_ * TILE16, hi, idesc_qk, 0u);
             };
             auto issue_pv = [&](int t_, int s_, bool acc) {
-                mma8_f16_ts<2048 / 16>(tmem + 256 + t_ * HD, tmem + t_ * BN, v_lo + s_ * TILE16, hi_pv, idesc_pv,
-                                       acc ? 1u : 0u);
+                mma8_f16_ts<32, 512, 128>(tmem + 256 + t_ * HD, tmem + t_ * BN, v_lo + s_ * TILE16, hi, idesc_pv,
+                                          acc ? 1u : 0u);
             };
             bool ok = true;
             for (int t = 0; t < nq && ok; ++t) ok = wait_thread(bar(Q_FULL + t), 0, wc);

@@ -384,12 +384,15 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint
 }
 
 // Arrive once on `bar` when every tcgen05 op this thread issued before has completed.
-// The 8 MMAs of a K = 128 contraction (K = 16 each) in one asm block, A and B from shared memory
-// in two 64-wide, 128-byte-swizzled halves of K that lie `half16` * 16 bytes apart: step k reads
-// at (k / 4) * half16 + (k % 4) * 2 (in 16-byte units) past the base descriptors, whose low
-// halves are a_lo / b_lo and whose high half is `hi`.  The first MMA overwrites D unless
-// `accumulate`; the others accumulate.
-template <uint32_t half16>
+// The 8 MMAs of a K = 128 contraction (K = 16 each) in one asm block, A and B from shared memory.
+// Step k reads A and B at (k / 4) * OFF_HI + (k % 4) * OFF_LO past their base descriptors, in
+// the descriptors' 16-byte address units: K-major 128-byte-swizzled operands whose 64-wide halves
+// of K lie h bytes apart take (h / 16, 2); MN-major ones with 2048 bytes per 16 rows of K take
+// (512, 128).  a_lo / b_lo are the base descriptors' low halves (address and leading offset),
+// `hi` their common high half (stride offset, version, swizzle): adding to the low half moves the
+// start address, with no carry out of its 14-bit field while addresses stay below 256 KB.  The
+// first MMA overwrites D unless `accumulate`; the others accumulate.
+template <uint32_t OFF_HI, uint32_t OFF_LO>
 __device__ __forceinline__ void mma8_f16_ss(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc,
                                             uint32_t accumulate) {
     asm volatile(
@@ -397,12 +400,6 @@ __device__ __forceinline__ void mma8_f16_ss(uint32_t d, uint32_t a_lo, uint32_t 
         "setp.ne.b32 p0, %5, 0;\n\tsetp.eq.b32 p1, %4, %4;\n\t"
         "mov.b64 a, {%1, %3};\n\tmov.b64 b, {%2, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p0;\n\t"
-        "add.u32 x, %1, 2;\n\tadd.u32 y, %2, 2;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
-        "add.u32 x, %1, 4;\n\tadd.u32 y, %2, 4;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
-        "add.u32 x, %1, 6;\n\tadd.u32 y, %2, 6;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
         "add.u32 x, %1, %6;\n\tadd.u32 y, %2, %6;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
         "add.u32 x, %1, %7;\n\tadd.u32 y, %2, %7;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
@@ -410,15 +407,21 @@ __device__ __forceinline__ void mma8_f16_ss(uint32_t d, uint32_t a_lo, uint32_t 
         "add.u32 x, %1, %8;\n\tadd.u32 y, %2, %8;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
         "add.u32 x, %1, %9;\n\tadd.u32 y, %2, %9;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, %10;\n\tadd.u32 y, %2, %10;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, %11;\n\tadd.u32 y, %2, %11;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, %12;\n\tadd.u32 y, %2, %12;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %4, p1;\n\t}" ::"r"(d),
-        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "n"(half16), "n"(half16 + 2),
-        "n"(half16 + 4), "n"(half16 + 6)
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "n"(OFF_LO), "n"(2 * OFF_LO),
+        "n"(3 * OFF_LO), "n"(OFF_HI), "n"(OFF_HI + OFF_LO), "n"(OFF_HI + 2 * OFF_LO), "n"(OFF_HI + 3 * OFF_LO)
         : "memory");
 }
-// The 8 MMAs of a K = 128 contraction with A from TMEM (a_tmem + 8 k: bf16 pairs, 16 elements
-// of K per 8 columns) and B from shared memory, step k at k * step16 (16-byte units) past the
-// base descriptor (low half b_lo, high half hi).
-template <uint32_t step16>
+// The 8 MMAs of a K = 128 contraction with A from TMEM (bf16 pairs, 8 columns per 16 elements of
+// K): step k reads A at column a_tmem + (k / 4) * A_HI + (k % 4) * 8 and B at (k / 4) * B_HI +
+// (k % 4) * B_LO past its base descriptor (low half b_lo, high half hi), as mma8_f16_ss.
+template <uint32_t A_HI, uint32_t B_HI, uint32_t B_LO>
 __device__ __forceinline__ void mma8_f16_ts(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t hi, uint32_t idesc,
                                             uint32_t accumulate) {
     asm volatile(
@@ -432,18 +435,25 @@ __device__ __forceinline__ void mma8_f16_ts(uint32_t d, uint32_t a_tmem, uint32_
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
         "add.u32 x, %2, %8;\n\tadd.u32 t, %1, 24;\n\tmov.b64 b, {x, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
-        "add.u32 x, %2, %9;\n\tadd.u32 t, %1, 32;\n\tmov.b64 b, {x, %3};\n\t"
+        "add.u32 x, %2, %9;\n\tadd.u32 t, %1, %13;\n\tmov.b64 b, {x, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
-        "add.u32 x, %2, %10;\n\tadd.u32 t, %1, 40;\n\tmov.b64 b, {x, %3};\n\t"
+        "add.u32 x, %2, %10;\n\tadd.u32 t, %1, %14;\n\tmov.b64 b, {x, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
-        "add.u32 x, %2, %11;\n\tadd.u32 t, %1, 48;\n\tmov.b64 b, {x, %3};\n\t"
+        "add.u32 x, %2, %11;\n\tadd.u32 t, %1, %15;\n\tmov.b64 b, {x, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t"
-        "add.u32 x, %2, %12;\n\tadd.u32 t, %1, 56;\n\tmov.b64 b, {x, %3};\n\t"
+        "add.u32 x, %2, %12;\n\tadd.u32 t, %1, %16;\n\tmov.b64 b, {x, %3};\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [t], b, %4, p1;\n\t}" ::"r"(d),
-        "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "n"(step16), "n"(2 * step16),
-        "n"(3 * step16), "n"(4 * step16), "n"(5 * step16), "n"(6 * step16), "n"(7 * step16)
+        "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "n"(B_LO), "n"(2 * B_LO), "n"(3 * B_LO),
+        "n"(B_HI), "n"(B_HI + B_LO), "n"(B_HI + 2 * B_LO), "n"(B_HI + 3 * B_LO), "n"(A_HI), "n"(A_HI + 8),
+        "n"(A_HI + 16), "n"(A_HI + 24)
         : "memory");
 }
+// Low and high halves of a shared-memory descriptor (sdesc_sw128).
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+    return static_cast<uint32_t>(sdesc_sw128(saddr, lbo_bytes, 1024));
+}
+__device__ __forceinline__ uint32_t sdesc_hi() { return static_cast<uint32_t>(sdesc_sw128(0, 16, 1024) >> 32); }
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
