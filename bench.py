@@ -31,10 +31,12 @@ import synth  # noqa: E402
 
 METRIC = "attention TFLOP/s (4*B*H*S^2*D fwd)"
 
-# DRAM bytes (read + write) of one launch of the dominant kernel from an ncu
-# capture (profiles/), per workload; None where the kernel changed since.
-TRAFFIC = {"wan14b_720p": 3.337e9, "train_480p_fwd_bwd": 3.809e9, "q8_720p": 1.936e9, "fp8_qkv_720p": 5.028e9,
-           "sparse8_720p": 3.429e9}
+# DRAM bytes (read + write) of one launch of the dominant kernel from an ncu capture of the
+# current kernel on a smaller case (one kernel, one launch), scaled to the workload by S*H;
+# absent where the kernel changed since its last capture.  The captures are summarised in
+# profiles/.
+TRAFFIC = {"wan14b_720p": 2.955e9, "train_480p_fwd_bwd": 3.582e9, "q8_720p": 1.594e9, "sparse8_720p": 2.918e9,
+           "fp8_qkv_720p": 5.028e9}
 
 
 def load_peaks():
