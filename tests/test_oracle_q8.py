@@ -4,7 +4,9 @@
   round to nearest even) on every value below the saturation point, plus the
   saturating closed form above it and a round trip through all 254 finite codes;
 * int8 block quantisation against closed forms (absmax maps to +-127, zero
-  block, ragged last block, block boundaries);
+  block, ragged last block, block boundaries), and its codes (from a product
+  with the block's fp32 reciprocal scale) against the textbook division by the
+  scale: at most one step apart, on a 1e-4 fraction of elements at most;
 * the diagnostic 8-bit simulation reduces to the dequantised V for S = 1 and
   stays within the quantisation error budget of the exact oracle;
 * the simulation's folded form (each block's V scale carried inside P) against
@@ -184,3 +186,19 @@ def test_q8_planted_fold_mistakes_are_caught(monkeypatch, kind):
     o_f, _ = q8.attn_fwd_q8_sim(q, k, v)
     o_b, _ = q8.attn_fwd_q8_blockwise(q, k, v)
     assert np.linalg.norm(o_f - o_b) / np.linalg.norm(o_b) > 1e-3
+
+
+def test_int8_codes_by_reciprocal_product_match_division_but_for_rare_ties():
+    # The quantiser forms its codes as rint(fp32(x * fp32(127 / absmax))); the textbook form is
+    # rint(x / (absmax / 127)).  Both round the same real quotient up to an fp32 rounding or two,
+    # so codes differ by at most one step and only where the quotient sits within an ulp of a
+    # half-integer: the reading of the pages' "absmax/127 scale" does not change the recipe.
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((1, 4096, 4, 128)).astype(np.float32)
+    codes, scale = q8.quant_int8(x)
+    amax = q8.block_absmax(x)
+    per = np.repeat(amax, 64, axis=2)[:, :, :4096].transpose(0, 2, 1)[:, :, :, None].astype(np.float64)
+    textbook = np.clip(np.rint(x.astype(np.float64) / (per / 127.0)), -127, 127)
+    diff = np.abs(codes.astype(np.int64) - textbook.astype(np.int64))
+    assert diff.max() <= 1
+    assert np.count_nonzero(diff) <= 1e-4 * diff.size
