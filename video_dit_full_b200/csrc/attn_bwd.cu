@@ -65,6 +65,11 @@ constexpr int SMEM_BYTES = SMEM_USED + 1024;
 constexpr int NTHREADS = 352;
 constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_RED = 10;
 constexpr int G_THREADS = 256;
+constexpr int G_WARPS = G_THREADS / 32;
+#ifndef WAN_BWD_WARP_ARRIVE
+#define WAN_BWD_WARP_ARRIVE 1         // the gradient warps' barriers count one arrival per warp
+#endif
+constexpr int G_ARRIVALS = WAN_BWD_WARP_ARRIVE ? G_WARPS : G_THREADS;
 constexpr uint32_t TMEM_COLS = 512;      // S^T | dP^T | dV | dK
 constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
 constexpr float LOG2E = 1.4426950408889634f;
@@ -72,6 +77,17 @@ constexpr float LOG2E = 1.4426950408889634f;
 #define WAN_BWD_POLY_PAIRS 2          // of every 8 pairs of exponentials in P, this many use exp2_poly3
 #endif
 constexpr int BWD_POLY_PAIRS = WAN_BWD_POLY_PAIRS;
+
+// A gradient warp's arrival on one of its barriers, after every lane's writes and fences: one
+// arrival per warp (lane 0, once the warp has converged) or one per thread.
+__device__ __forceinline__ void g_arrive(uint32_t bar, int lane) {
+    if (WAN_BWD_WARP_ARRIVE) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar);
+    } else {
+        mbar_arrive(bar);
+    }
+}
 
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -138,17 +154,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
         }
         mbar_init(bar(S_FULL), 1);
         mbar_init(bar(DP_FULL), 1);
-        mbar_init(bar(P_READY), G_THREADS);
+        mbar_init(bar(P_READY), G_ARRIVALS);
         mbar_init(bar(DV_DONE), 1);
-        mbar_init(bar(DS_READY), G_THREADS);     // dS^T in TMEM (dK may start)
-        mbar_init(bar(DS_SMEM), G_THREADS);      // dS^T in shared memory (dQ may start)
+        mbar_init(bar(DS_READY), G_ARRIVALS);     // dS^T in TMEM (dK may start)
+        mbar_init(bar(DS_SMEM), G_ARRIVALS);      // dS^T in shared memory (dQ may start)
         mbar_init(bar(DQ_FULL), 1);
-        mbar_init(bar(DQ_DRAINED), G_THREADS);
+        mbar_init(bar(DQ_DRAINED), G_ARRIVALS);
         mbar_init(bar(FINAL), 1);
         mbar_init(bar(DRAIN), 1);
-        mbar_init(bar(STAGED), G_THREADS);
+        mbar_init(bar(STAGED), G_ARRIVALS);
         mbar_init(bar(RED_DONE), 1);
-        mbar_init(bar(EPI_STAGED), G_THREADS);
+        mbar_init(bar(EPI_STAGED), G_ARRIVALS);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -344,7 +360,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(P_READY));
+            g_arrive(bar(P_READY), lane);
 
             ok = wait_warp(bar(DP_FULL), i & 1, wc);
             if (!ok) break;
@@ -357,15 +373,17 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const float d0 = pr[2 * e] * (__uint_as_float(dp[2 * e]) - s_del[2 * e]);
-                    const float d1 = pr[2 * e + 1] * (__uint_as_float(dp[2 * e + 1]) - s_del[2 * e + 1]);
-                    dsp[e] = pack_bf16x2(d0, d1);
+                    // dS = P (dP - D), a pair at a time
+                    const float2 dd = fsub2(make_float2(__uint_as_float(dp[2 * e]), __uint_as_float(dp[2 * e + 1])),
+                                            make_float2(s_del[2 * e], s_del[2 * e + 1]));
+                    const float2 ds = fmul2(make_float2(pr[2 * e], pr[2 * e + 1]), dd);
+                    dsp[e] = pack_bf16x2(ds.x, ds.y);
                 }
             }
             tmem_st32(tDP, dsp);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(DS_READY));
+            g_arrive(bar(DS_READY), lane);
             // dS^T row j, queries cb..cb+63 -> the 128-byte swizzled row j of half hq, in dO's
             // buffer: only once dV (the last reader of dO) is done
             ok = wait_warp(bar(DV_DONE), i & 1, wc);
@@ -376,7 +394,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 *reinterpret_cast<uint4*>(half_row + ((ch ^ (j & 7)) * 16)) =
                     make_uint4(dsp[4 * ch], dsp[4 * ch + 1], dsp[4 * ch + 2], dsp[4 * ch + 3]);
             fence_async_smem();
-            mbar_arrive(bar(DS_SMEM));
+            g_arrive(bar(DS_SMEM), lane);
 
             ok = wait_warp(bar(DQ_FULL), i & 1, wc);
             if (!ok) break;
@@ -394,9 +412,9 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                 for (int e = 0; e < 32; ++e) stage[(cb + q * 32 + e) * HD + j] = __uint_as_float(v[e]);
             }
             tc_fence_before();
-            mbar_arrive(bar(DQ_DRAINED));
+            g_arrive(bar(DQ_DRAINED), lane);
             fence_async_smem();
-            mbar_arrive(bar(STAGED));
+            g_arrive(bar(STAGED), lane);
         }
         if (ok) ok = wait_warp(bar(FINAL), 0, wc);
         if (ok && p.nsplit > 1) {
@@ -422,7 +440,7 @@ bwd_main_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
                     }
                 }
                 fence_async_smem();
-                mbar_arrive(bar(EPI_STAGED));
+                g_arrive(bar(EPI_STAGED), lane);
             }
         } else if (ok) {
             tc_fence_after();
