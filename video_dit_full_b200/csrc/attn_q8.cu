@@ -170,25 +170,10 @@ constexpr float P_SCALE = 224.f;
 constexpr float LOG2_P_SCALE = 7.807354922057604f;
 
 // S (int32) = Q8 K8^T: Q [128 rows][128 bytes], K [64 rows][128 bytes], both K-major with the
-// 128-byte swizzle, K = 32 per MMA.
-__device__ __forceinline__ void issue_qk8(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem, uint32_t idesc) {
-#pragma unroll
-    for (int kk = 0; kk < HD / 32; ++kk)
-        mma_i8_ss(d_tmem, sdesc_sw128(q_smem + kk * 32, 16, 1024), sdesc_sw128(k_smem + kk * 32, 16, 1024),
-                  idesc, kk > 0 ? 1u : 0u);
-}
-
-// O (fp32, TMEM) += P8 V8: P8 in TMEM (4 e4m3 per column, 16 columns for the 64 keys), V8
-// [key][d] MN-major (one 128-byte swizzle atom spans all 128 d), 32 keys per MMA.  The tensor
-// core's fp32 accumulator carries the sum across every 64-key block; each block's V scale is
-// already in P8.
-__device__ __forceinline__ void issue_pv8(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc,
-                                          bool accumulate) {
-#pragma unroll
-    for (int kk = 0; kk < BN / 32; ++kk)
-        mma_f8_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(v_smem + kk * 4096, 16, 1024), idesc,
-                  (accumulate || kk > 0) ? 1u : 0u);
-}
+// 128-byte swizzle, K = 32 per MMA (mma4_i8_ss).  O (fp32, TMEM) += P8 V8: P8 in TMEM (4 e4m3 per
+// column, 16 columns for the 64 keys), V8 [key][d] MN-major (one 128-byte swizzle atom spans all
+// 128 d), 32 keys per MMA (mma2_f8_ts).  The tensor core's fp32 accumulator carries the sum
+// across every 64-key block; each block's V scale is already in P8.
 
 __global__ void __launch_bounds__(NTHREADS, 1)
 q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -293,14 +278,22 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
         if (lane == 0 && t < nq) {
             const uint32_t idesc_qk = make_idesc(2, 1, 1, 0, 0, BM, BN);   // s32 <- s8 x s8
             const uint32_t idesc_pv = make_idesc(1, 0, 0, 0, 1, BM, HD);   // f32 <- e4m3 x e4m3, V MN-major
-            const uint32_t tq = sQ + t * TQ8, to = tmem + T_O + t * HD;
+            const uint32_t to = tmem + T_O + t * HD;
             auto sbuf = [&](int j) { return tmem + static_cast<uint32_t>((2 * t + (j & 1)) * BN); };
+            // descriptor halves built once: Q of this tile, K and V of stage 0 (a stage is TKV8 / 16
+            // address units further on); one common high half
+            const uint32_t hi = sdesc_hi();
+            const uint32_t q_lo = sdesc_lo(sQ + t * TQ8, 16), k_lo = sdesc_lo(sK, 16), v_lo = sdesc_lo(sV, 16);
+            auto issue_qk8 = [&](int j, int st) { mma4_i8_ss(sbuf(j), q_lo, k_lo + st * (TKV8 / 16), hi, idesc_qk); };
+            auto issue_pv8 = [&](int j, int st) {
+                mma2_f8_ts(to, sbuf(j), v_lo + st * (TKV8 / 16), hi, idesc_pv, j > 0 ? 1u : 0u);
+            };
             bool ok = wait_thread(bar(Q_FULL + t), 0, wc);
             for (int j = 0; j < 2 && j < nkv && ok; ++j) {
                 ok = wait_thread(bar(KV_FULL + j), 0, wc);
                 if (!ok) break;
                 tc_fence_after();
-                issue_qk8(sbuf(j), tq, sK + j * TKV8, idesc_qk);
+                issue_qk8(j, j);
                 mma_commit(bar(S_FULL + 2 * t + j));
             }
             for (int j = 0; j < nkv && ok; ++j) {
@@ -312,12 +305,12 @@ q8_attn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ 
                 if (ok) ok = wait_thread(bar(P_FULL + 2 * t + (j & 1)), (j >> 1) & 1, wc);
                 if (!ok) break;
                 tc_fence_after();
-                issue_pv8(to, sbuf(j), sV + s * TKV8, idesc_pv, j > 0);
+                issue_pv8(j, s);
                 mma_commit(bar(KV_EMPTY + s));               // after K(j)'s and V(j)'s last readers
                 if (j + 2 == nkv) mma_commit(bar(PV_LAST + t));
                 if (j + 1 == nkv) mma_commit(bar(O_FINAL + t));
                 if (next) {
-                    issue_qk8(sbuf(j), tq, sK + s2 * TKV8, idesc_qk);
+                    issue_qk8(j, s2);
                     mma_commit(bar(S_FULL + 2 * t + (j & 1)));
                 }
             }

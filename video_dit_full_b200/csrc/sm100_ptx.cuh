@@ -448,6 +448,39 @@ __device__ __forceinline__ void mma8_f16_ts(uint32_t d, uint32_t a_tmem, uint32_
         "n"(A_HI + 16), "n"(A_HI + 24)
         : "memory");
 }
+// The 4 MMAs of an int8 K = 128 contraction (K = 32 each) in one asm block, A and B K-major with
+// 128-byte rows in shared memory: step k reads both at k * 32 bytes past the base descriptors
+// (low halves a_lo / b_lo, common high half hi).  The first MMA overwrites D.
+__device__ __forceinline__ void mma4_i8_ss(uint32_t d, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t.reg .b32 x, y;\n\t.reg .b64 a, b;\n\t"
+        "setp.ne.b32 p0, %4, %4;\n\tsetp.eq.b32 p1, %4, %4;\n\t"
+        "mov.b64 a, {%1, %3};\n\tmov.b64 b, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], a, b, %4, p0;\n\t"
+        "add.u32 x, %1, 2;\n\tadd.u32 y, %2, 2;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, 4;\n\tadd.u32 y, %2, 4;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], a, b, %4, p1;\n\t"
+        "add.u32 x, %1, 6;\n\tadd.u32 y, %2, 6;\n\tmov.b64 a, {x, %3};\n\tmov.b64 b, {y, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], a, b, %4, p1;\n\t}" ::"r"(d),
+        "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc)
+        : "memory");
+}
+// The 2 MMAs of an e4m3 K = 64 contraction (K = 32 each) with A from TMEM (a_tmem, a_tmem + 8)
+// and B MN-major in shared memory, 4096 bytes per 32 rows of K (base descriptor low half b_lo,
+// high half hi).  The first MMA accumulates only if `accumulate`.
+__device__ __forceinline__ void mma2_f8_ts(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t hi, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t.reg .b32 x, t;\n\t.reg .b64 b;\n\t"
+        "setp.ne.b32 p0, %5, 0;\n\tsetp.eq.b32 p1, %4, %4;\n\t"
+        "mov.b64 b, {%2, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], b, %4, p0;\n\t"
+        "add.u32 x, %2, 256;\n\tadd.u32 t, %1, 8;\n\tmov.b64 b, {x, %3};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [t], b, %4, p1;\n\t}" ::"r"(d),
+        "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // Low and high halves of a shared-memory descriptor (sdesc_sw128).
 __device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo_bytes) {
     return static_cast<uint32_t>(sdesc_sw128(saddr, lbo_bytes, 1024));
