@@ -35,7 +35,7 @@ METRIC = "attention TFLOP/s (4*B*H*S^2*D fwd)"
 # current kernel on a smaller case (one kernel, one launch), scaled to the workload by S*H;
 # absent where the kernel changed since its last capture.  The captures are summarised in
 # profiles/.
-TRAFFIC = {"wan14b_720p": 2.955e9, "train_480p_fwd_bwd": 3.714e9, "q8_720p": 1.594e9, "sparse8_720p": 2.918e9,
+TRAFFIC = {"wan14b_720p": 2.955e9, "train_480p_fwd_bwd": 3.714e9, "q8_720p": 1.594e9, "sparse8_720p": 2.927e9,
            "fp8_qkv_720p": 5.028e9}
 
 
@@ -521,8 +521,8 @@ class SparsePath:
         size = np.minimum(64, w.S - 64 * np.arange(nb)).astype(np.float64)
         self.flop = float(4.0 * w.D * np.einsum("bhij,i,j->", self.mask_host.astype(np.float64), size, size))
         self.dense_flop = w.fwd_flop
-        m4 = np.pad(self.mask_host, ((0, 0), (0, 0), (0, (-nb) % 4), (0, 0)))
-        union = m4.reshape(w.B, w.H, -1, 4, nb).max(axis=3)
+        m2 = np.pad(self.mask_host, ((0, 0), (0, 0), (0, nb % 2), (0, 0)))   # 128-row Q tiles
+        union = m2.reshape(w.B, w.H, -1, 2, nb).max(axis=3)
         self.union_frac = float(union.mean())
         self.host_in = [pinned(x[n]) for n in ("q", "k", "v")]
         self.dev_in = [t.to(dev) for t in self.host_in]
@@ -534,8 +534,8 @@ class SparsePath:
                               device=dev)
         self.outs = [self.o, self.lse]
         self.dominant_flop = self.flop
-        self.kernel = ("wan::sparse::attn_fwd_sparse_kernel (with its per-tile key-block list kernel: one "
-                       "wan_attn_fwd_block_sparse)")
+        self.kernel = ("wan::sparse::pair::attn_fwd_sparse_pair_kernel (with its per-tile key-block list "
+                       "kernel: one wan_attn_fwd_block_sparse)")
         self.launches_per_step = 2
         self.peak_key, self.dtype = "bf16", "bf16"
         self.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]

@@ -16,8 +16,9 @@ struct FwdParams {
     int Skv;                    // key / value tokens (= S for self-attention)
     // block-sparse forward only: 64 x 64 block mask uint8 [B, H, nqb, nkb], and per 128-row Q
     // tile (2 query blocks) the ascending list of key blocks either attends
-    // (kv_list [B, H, nctas, nkb] int32, nctas = the number of Q tiles) with its length
-    // (kv_count [B, H, nctas])
+    // (kv_list [B, H, nctas, nkb] int32, nctas = the number of Q tiles; each entry the key block
+    // with bit 30 set if the tile's first query block attends it, bit 31 if the second does)
+    // with its length (kv_count [B, H, nctas])
     const uint8_t* mask;
     const int* kv_list;
     const int* kv_count;
@@ -80,10 +81,11 @@ int configure_smem(const void* kernel, int bytes);
 // `to`: a map over O with the layout and box of tq (the epilogue TMA-stores O through it).
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                const FwdParams& p, cudaStream_t stream);
-// Forward with one CTA per 128-row Q tile (p.nctas = the number of Q tiles), 64-key steps; tk64 /
-// tv64 are K / V maps with 64-token boxes.  Block-sparse (p.kv_list set): builds each tile's
-// key-block list in p.kv_list / p.kv_count (device workspace) from p.mask, then runs the kernel
-// over the lists.  p.kv_list null: every key block, no mask.
+// Forward with one CTA per 128-row Q tile (p.nctas = the number of Q tiles); tk64 / tv64 are
+// K / V maps with 64-token boxes.  Block-sparse (p.kv_list set): builds each tile's
+// key-block list in p.kv_list / p.kv_count (device workspace) from p.mask, then runs the
+// pair-step kernel over the lists.  p.kv_list null: every key block, no mask, on the per-tile
+// kernel with 64-key steps.
 int launch_fwd_tiles(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv64, const CUtensorMap& to,
                      const FwdParams& p, cudaStream_t stream);
 
