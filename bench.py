@@ -316,7 +316,7 @@ class Path:
             self.flop = w.fwd_flop
             self.dominant_flop = w.fwd_flop
             if w.cross and w.kv_len != w.S and w.kv_len <= 1024:   # the short-key cross forward's kernel
-                self.kernel = "wan::sparse::pair::attn_fwd_pair_kernel<true>, every key block (wan_attn_cross_fwd)"
+                self.kernel = "wan::sparse::pair::attn_fwd_pair_kernel<true, true>, every key block (wan_attn_cross_fwd)"
             else:
                 self.kernel = "wan::fwd::attn_fwd_kernel" + (" (wan_attn_cross_fwd)" if w.cross else "")
             self.launches_per_step = 1
@@ -534,7 +534,7 @@ class SparsePath:
                               device=dev)
         self.outs = [self.o, self.lse]
         self.dominant_flop = self.flop
-        self.kernel = ("wan::sparse::pair::attn_fwd_pair_kernel<false> (with its per-tile key-block list "
+        self.kernel = ("wan::sparse::pair::attn_fwd_pair_kernel<false, false> (with its per-tile key-block list "
                        "kernel: one wan_attn_fwd_block_sparse)")
         self.launches_per_step = 2
         self.peak_key, self.dtype = "bf16", "bf16"
