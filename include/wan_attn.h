@@ -67,8 +67,10 @@ typedef enum {
  *   lse     : out, fp32 [B, H, S], natural-log log-sum-exp of the scaled
  *             scores of each query row (the backward's input); not NULL.
  *   B, S, H : >= 1, with B*S*H*D < 2^40;  D : must be 128.
- * Accumulation is fp32 (scores, running max and sum, and O).  Returns
- * WAN_ATTN_OK once the kernel is enqueued.
+ * Accumulation is fp32 (scores, running max and sum, and O); P = 2^(s - m)
+ * is rounded to bf16 for P V.  Of every 16 exponentials 14 come from the
+ * hardware exp2 and 2 from a degree-3 polynomial (relative error 7.5e-5).
+ * Returns WAN_ATTN_OK once the kernel is enqueued.
  */
 WAN_ATTN_API int wan_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                  int B, int S, int H, int D, void* stream);

@@ -51,7 +51,7 @@ constexpr int NTHREADS = 320;
 constexpr uint32_t TMEM_COLS = 512;            // S0 S1 O0 O1, 128 columns each
 constexpr float RESCALE_THRESHOLD = 8.0f;      // log2 units: keep a stale max while p <= 2^8
 #ifndef WAN_FWD_POLY_PAIRS
-#define WAN_FWD_POLY_PAIRS 0          // of every 8 pairs of exponentials, this many use exp2_poly3_x2
+#define WAN_FWD_POLY_PAIRS 1          // of every 8 pairs of exponentials, this many use exp2_poly3_x2
 #endif
 constexpr int FWD_POLY_PAIRS = WAN_FWD_POLY_PAIRS;
 
