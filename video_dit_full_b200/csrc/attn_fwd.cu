@@ -244,8 +244,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__
             }
             // P = 2^(s c - m) in packed pairs, the row sum in four independent packed accumulators.
             // Of every 8 pairs FWD_POLY_PAIRS come from the degree-3 polynomial on the FMA pipe and
-            // the rest from the MUFU (none by default: the polynomial's extra instructions slow the
-            // MMA issuer that shares a sub-partition with the softmax warps more than they save).
+            // the rest from the MUFU (1 by default; more of them slow the MMA issuer, which shares
+            // a sub-partition with two softmax warps, by more than they save).
             const float2 c2 = make_float2(c, c), n2 = make_float2(-m_ref, -m_ref);
             float2 acc[4];
 #pragma unroll
