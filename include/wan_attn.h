@@ -120,8 +120,9 @@ WAN_ATTN_API int wan_attn_bwd(const void* q, const void* k, const void* v, const
  * passes the padded embedding, as the 512-token condition is).  Other
  * conventions, precision and errors as wan_attn_fwd; wan_attn_cross_fwd with
  * Skv = Sq and the same pointers computes what wan_attn_fwd does, bit for bit.
- * With Sq != Skv <= 1024 the call takes 64 keys per step (one CTA per
- * 128-query tile, two per SM), so its rounding differs from a 128-key step's.
+ * With Sq != Skv <= 1024 the call runs one CTA per 128-query tile, two per SM,
+ * in 128-key steps with every exponential from the hardware exp2, so its
+ * rounding differs slightly from wan_attn_fwd's.
  */
 WAN_ATTN_API int wan_attn_cross_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                                     int Sq, int Skv, int H, int D, void* stream);
@@ -170,9 +171,11 @@ WAN_ATTN_API int wan_attn_cross_bwd(const void* q, const void* k, const void* v,
  *     lists of attended key blocks (int32 [B, H, ceil(Sq/128), ceil(Skv/64)])
  *     and their lengths, built on the device by this call.
  * Work: a CTA covers one 128-row Q tile (2 query blocks) and steps through
- * the union of the key blocks its 2 query blocks attend, one 64-key block per
- * step; each row keeps only its own query block's blocks.  Other conventions
- * as wan_attn_fwd.
+ * the union of the key blocks its 2 query blocks attend, two listed blocks
+ * (128 keys) per step; each row keeps only its own query block's blocks, and
+ * a query block that skips one of a step's blocks gets P = 0 for its 64 keys.
+ * Every exponential comes from the hardware exp2.  Other conventions as
+ * wan_attn_fwd.
  */
 WAN_ATTN_API size_t wan_attn_fwd_block_sparse_workspace_size(int B, int Sq, int Skv, int H, int D);
 WAN_ATTN_API int wan_attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
