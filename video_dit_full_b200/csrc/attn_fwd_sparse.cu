@@ -87,6 +87,9 @@ struct Cfg {
     static constexpr int SMEM_BYTES = OFF_ABORT + 8 + 1024;
     static constexpr uint32_t T_O = NBUF * BN;
     static constexpr uint32_t TMEM_COLS = T_O + HD;
+    static_assert(K_STAGES <= 3 && V_STAGES <= 3, "the producers track up to three stages per ring");
+    static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM is allocated in powers of two");
+    static_assert(SMEM_BYTES <= 232448 / MIN_CTAS, "shared memory for MIN_CTAS CTAs per SM");
 };
 constexpr int WARP_TMA_K = 4, WARP_PV = 5, WARP_TMA_V = 6, WARP_QK = 7;   // sparse roles; dense: 4 TMA, 5 MMA
 
