@@ -120,3 +120,52 @@ def test_tiles_that_need_one_half_or_start_late():
         else:
             mask[0, 1, qb, :3] = 1
     check(x, mask)
+
+
+def tile_lists_from_mask(mask):
+    """Each 128-row Q tile's ascending union of the key blocks its two query blocks attend, one
+    int32 entry per block: the block index, bit 30 set if the first query block attends it, bit 31
+    if the second does; and the union's length.  Built from the mask alone."""
+    B, H, nqb, nkb = mask.shape
+    ntiles = (nqb + 1) // 2
+    lists = np.zeros((B, H, ntiles, nkb), dtype=np.uint32)
+    counts = np.zeros((B, H, ntiles), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for t in range(ntiles):
+                r0 = mask[b, h, 2 * t] != 0
+                r1 = mask[b, h, 2 * t + 1] != 0 if 2 * t + 1 < nqb else np.zeros(nkb, dtype=bool)
+                kb = np.nonzero(r0 | r1)[0]
+                entries = kb.astype(np.uint32) | (r0[kb].astype(np.uint32) << 30) | (r1[kb].astype(np.uint32) << 31)
+                lists[b, h, t, :kb.size] = entries
+                counts[b, h, t] = kb.size
+    return lists, counts
+
+
+@pytest.mark.parametrize("Sq,Skv,keep", [(1300, 900, 0.3), (65, 64, 1.0), (4100, 333, 0.125)])
+def test_tile_lists_in_the_workspace_are_exact(Sq, Skv, keep):
+    # Integer work: the per-tile lists the call builds in its workspace must equal the ones built
+    # from the mask on the host, entry for entry (the workspace is int32 lists [B, H, ntiles, nkb]
+    # then, 256-byte aligned, the lengths [B, H, ntiles]; list entries past a length are unused).
+    import torch
+    import video_dit_full_b200 as wa
+    B, H = 2, 3
+    x = inputs_for_cross(B, Sq, Skv, H, seed=Sq)
+    mask = synth.block_mask(B, H, bs.blocks(Sq), bs.blocks(Skv), keep, seed=Skv)
+    q, k, v = (to_device(x[n]) for n in "qkv")
+    ws = torch.zeros(wa.block_sparse_workspace_size(B, Sq, Skv, H), dtype=torch.uint8, device="cuda")
+    wa.fwd_block_sparse(q, k, v, torch.from_numpy(mask).cuda(), workspace=ws)
+    wa.check_status()
+    want_lists, want_counts = tile_lists_from_mask(mask)
+    ntiles, nkb = want_lists.shape[2], want_lists.shape[3]
+    list_bytes = B * H * ntiles * nkb * 4
+    raw = ws.cpu().numpy()
+    got_lists = raw[:list_bytes].view(np.uint32).reshape(B, H, ntiles, nkb)
+    off = (list_bytes + 255) // 256 * 256
+    got_counts = raw[off:off + B * H * ntiles * 4].view(np.int32).reshape(B, H, ntiles)
+    assert np.array_equal(got_counts, want_counts)
+    for b in range(B):
+        for h in range(H):
+            for t in range(ntiles):
+                n = want_counts[b, h, t]
+                assert np.array_equal(got_lists[b, h, t, :n], want_lists[b, h, t, :n]), (b, h, t)
