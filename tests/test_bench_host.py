@@ -39,3 +39,16 @@ def test_roofline_peak_per_kernel():
     gemm = object.__new__(bench.GemmPath)
     gemm.peak_key = "fp8"
     assert bench.peak_for(gemm, peaks, {"fp8_e4m3_tflops": 3000.0, "int8_tops": 2000.0})[0] == 3000.0
+
+
+def test_union_fraction_of_the_block_sparse_tiles():
+    import numpy as np
+    import bench
+    m = np.zeros((1, 1, 3, 4), dtype=np.uint8)
+    m[0, 0, 0, [0, 2]] = 1            # tile 0: query blocks 0 and 1 -> union {0, 2, 3}
+    m[0, 0, 1, [2, 3]] = 1
+    m[0, 0, 2, [1]] = 1               # tile 1: query block 2 alone -> {1}
+    assert bench.union_fraction(m) == pytest.approx((3 + 1) / (2 * 4))
+    rng = np.random.default_rng(0)    # independent rows at density d: 1 - (1 - d)^2
+    r = (rng.random((1, 8, 64, 4096)) < 0.125).astype(np.uint8)
+    assert bench.union_fraction(r) == pytest.approx(1 - 0.875 ** 2, abs=3e-3)
