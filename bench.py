@@ -502,6 +502,14 @@ class GemmPath:
         self.host_in, self.host_out = other.host_in, other.host_out
 
 
+def union_fraction(mask):
+    """Fraction of (Q tile, key block) pairs a CTA computes: each 128-row Q tile walks the union of
+    the key blocks its two 64-row query blocks attend (a short last tile has one)."""
+    nqb = mask.shape[2]
+    m2 = np.pad(mask, ((0, 0), (0, 0), (0, nqb % 2), (0, 0)))
+    return float(m2.reshape(mask.shape[0], mask.shape[1], -1, 2, mask.shape[3]).max(axis=3).mean())
+
+
 class SparsePath:
     """Block-sparse attention: one wan_attn_fwd_block_sparse over a seeded 64 x 64 block mask.
     `flop` counts only the allowed blocks (4 * D * |query block| * |key block| each); the
@@ -521,9 +529,7 @@ class SparsePath:
         size = np.minimum(64, w.S - 64 * np.arange(nb)).astype(np.float64)
         self.flop = float(4.0 * w.D * np.einsum("bhij,i,j->", self.mask_host.astype(np.float64), size, size))
         self.dense_flop = w.fwd_flop
-        m2 = np.pad(self.mask_host, ((0, 0), (0, 0), (0, nb % 2), (0, 0)))   # 128-row Q tiles
-        union = m2.reshape(w.B, w.H, -1, 2, nb).max(axis=3)
-        self.union_frac = float(union.mean())
+        self.union_frac = union_fraction(self.mask_host)
         self.host_in = [pinned(x[n]) for n in ("q", "k", "v")]
         self.dev_in = [t.to(dev) for t in self.host_in]
         self.mask = torch.from_numpy(self.mask_host).to(dev)
