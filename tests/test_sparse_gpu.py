@@ -1,8 +1,10 @@
 """Parity of the block-sparse forward (wan_attn_fwd_block_sparse, through the C ABI) with the oracle
 (oracle/block_sparse.py): the bf16 forward's bars (O max-abs 1e-2 and rel-Frobenius 5e-3, LSE
 1e-3) on the rows that attend something; rows that attend nothing must be exactly O = 0,
-LSE = -inf.  An all-ones mask must agree with wan_attn_fwd to rounding (the two kernels take
-the keys in steps of 64 and 128, so their online softmax rescales at different points)."""
+LSE = -inf.  An all-ones mask must agree with wan_attn_fwd to rounding (the two kernels mix
+their exponentials differently and rescale at different points).  The per-tile key-block lists
+the call builds in its workspace must equal, entry for entry, the lists built on the host from the
+mask (integer work: bit-exact)."""
 import numpy as np
 import pytest
 
