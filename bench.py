@@ -840,7 +840,10 @@ def run_ours(args, w):
                        "l2": "inputs (%.2f GB) exceed the 126 MB L2; no flush" % in_gb},
             "gpu_launches": args.steps * path.launches_per_step,
             **({"sparse": {"keep": w.sparse_keep, "union_fraction_computed": path.union_frac,
-                           "dense_equivalent_tflops": whole_job_tflops(world, path.dense_flop, args.steps, total_ms)}}
+                           "dense_equivalent_tflops": whole_job_tflops(world, path.dense_flop, args.steps, total_ms),
+                           # the rate of the tensor work the tiles do: every key block of a tile's union
+                           "union_tflops": whole_job_tflops(world, path.union_frac * path.dense_flop, args.steps,
+                                                            total_ms)}}
                if w.sparse_keep else {}),
             "roofline": roofline_of(path, w, t, peaks, p8),
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": path.h2d_bytes,
