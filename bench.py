@@ -35,7 +35,7 @@ METRIC = "attention TFLOP/s (4*B*H*S^2*D fwd)"
 # current kernel on a smaller case (one kernel, one launch), scaled to the workload by S*H;
 # absent where the kernel changed since its last capture.  The captures are summarised in
 # profiles/.
-TRAFFIC = {"wan14b_720p": 2.948e9, "train_480p_fwd_bwd": 3.714e9, "q8_720p": 1.594e9, "sparse8_720p": 2.927e9,
+TRAFFIC = {"wan14b_720p": 2.948e9, "train_480p_fwd_bwd": 3.714e9, "q8_720p": 1.599e9, "sparse8_720p": 2.927e9,
            "fp8_qkv_720p": 5.028e9}
 
 
